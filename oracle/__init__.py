@@ -1,0 +1,20 @@
+"""CPU oracle for the DFlash draft cycle — TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, float64 NumPy restatement of what one draft cycle computes,
+written from the DFlash pages and kept free of any blocking, fusion or
+reordering beyond what the definitions state. It shares no code with the CUDA
+path and never imports it. Only the test-suite, the smoke check and the
+benchmark's CPU-baseline leg may use it; the product path must not.
+
+Modules
+  dflash  -- feature fusion + KV injection, the block drafter, greedy verify
+  target  -- a tiny causal target model, greedy autoregressive decoding and the
+             speculative loop (for the lossless check)
+
+Parity status per function (what pins each one, see tests/test_oracle_*.py):
+  rms_norm, silu, apply_rope, block_attention, drafter_layer, inject,
+  draft_block                 pinned (closed forms, invariants, library routines)
+  greedy_argmax, verify       pinned (brute force, hand-worked golden cases)
+  TinyTarget, greedy_decode,
+  spec_generate               pinned (library decoder, lossless invariant)
+"""
