@@ -1,0 +1,689 @@
+// Host side of the C ABI (include/dflash.h): validation, workspace, TMA
+// descriptors, GEMM planning and the launch sequence of inject / draft.
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <tuple>
+#include <vector>
+
+#include "../../include/dflash.h"
+#include "gemm.cuh"
+#include "kernels.cuh"
+
+using namespace dfl;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kCountersPerSite = 4096;
+constexpr int kNumSites = 128;
+constexpr size_t kPartialFloats = (size_t)24 << 20;   // split-K partials: 96 MB
+constexpr int kAttnTargetCtas = 296;                   // 2 CTAs per SM on 148 SMs
+
+enum Site { SITE_FC = 0, SITE_KV = 1, SITE_LM = 4, SITE_LAYER0 = 8 };
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+enum ProfKind { PK_GEMM_TC = 0, PK_GEMM_SIMT, PK_ATTN, PK_EMBED_NORM, PK_RMSNORM, PK_ARGMAX, PK_COPY, PK_COUNT };
+const char* const kProfNames[PK_COUNT] = {"gemm_tc", "gemm_simt", "attention", "embed_norm",
+                                          "rmsnorm", "argmax_finalize", "hidden_copy"};
+
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double bytes, flops;
+};
+
+}  // namespace
+
+struct dflash_ctx {
+  dflash_config cfg;
+  bool bf16 = false;
+  bool force_simt = false;
+  bool use_pdl = false;
+  int num_sms = 148;
+  const void* fc = nullptr;
+  const void* embed = nullptr;
+  const void* lm_head = nullptr;
+  const float* final_norm = nullptr;
+  std::vector<const float*> attn_norm, mlp_norm;
+  std::vector<const void*> wq, wk, wv, wo, wg, wu, wd;
+  // workspace
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  float* x = nullptr;
+  void* h = nullptr;
+  void* q = nullptr;
+  void* kb = nullptr;
+  void* vb = nullptr;
+  void* ao = nullptr;
+  void* act = nullptr;
+  void* c = nullptr;
+  float* partials = nullptr;
+  int* counters = nullptr;
+  unsigned long long* keys = nullptr;
+  float* att_o = nullptr;
+  float* att_m = nullptr;
+  float* att_l = nullptr;
+  size_t att_rows = 0;   // capacity in (split, row) pairs
+  int* status = nullptr;
+  EncodeTiledFn encode = nullptr;
+  bool prof = false;
+  std::vector<ProfRec> recs;
+  std::map<std::tuple<const void*, long long, long long, long long, int>, CUtensorMap> maps;
+};
+
+namespace {
+
+int q_dim(const dflash_config& c) { return c.n_q_heads * c.head_dim; }
+int kv_dim(const dflash_config& c) { return c.n_kv_heads * c.head_dim; }
+size_t esize(const dflash_ctx* x) { return x->bf16 ? 2 : 4; }
+
+// A failed CUDA call is reported on stderr with the runtime's message, then as DFLASH_ERR_CUDA.
+dflash_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return DFLASH_OK;
+  std::fprintf(stderr, "dflash: %s: %s\n", where, cudaGetErrorString(e));
+  return DFLASH_ERR_CUDA;
+}
+
+// Brackets one launch with CUDA events when profiling is on.
+struct ProfScope {
+  dflash_ctx* ctx;
+  cudaStream_t st;
+  ProfRec rec{};
+  bool on;
+  ProfScope(dflash_ctx* c, int kind, cudaStream_t s, double bytes, double flops) : ctx(c), st(s), on(c->prof) {
+    if (!on) return;
+    rec.kind = kind;
+    rec.bytes = bytes;
+    rec.flops = flops;
+    cudaEventCreate(&rec.a);
+    cudaEventCreate(&rec.b);
+    cudaEventRecord(rec.a, st);
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(rec.b, st);
+    ctx->recs.push_back(rec);
+  }
+};
+
+bool get_map(dflash_ctx* ctx, const void* ptr, long long rows, long long K, long long ld, int box_rows,
+             CUtensorMap* out) {
+  auto key = std::make_tuple(ptr, rows, K, ld, box_rows);
+  auto it = ctx->maps.find(key);
+  if (it != ctx->maps.end()) {
+    *out = it->second;
+    return true;
+  }
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = ctx->encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  if (ctx->maps.size() > 4096) ctx->maps.clear();
+  ctx->maps[key] = m;
+  *out = m;
+  return true;
+}
+
+struct GemmSpec {
+  const void* x = nullptr;
+  int ldx = 0, M = 0, K = 0;
+  int n_seg = 0;
+  const void* w[kMaxSeg] = {};
+  int seg_rows[kMaxSeg] = {};
+  bool paired = false;
+  int site = 0;
+  EpiParams epi{};
+};
+
+int pow2_at_least(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
+  EpiParams& e = g.epi;
+  e.status = ctx->status;
+  e.out_bf16 = ctx->bf16 ? 1 : 0;
+  int n_tiles = 0;
+  if (g.paired) {
+    n_tiles = g.seg_rows[0] / (kTileN / 2);
+    e.n_seg = 1;
+    e.seg_tile_begin[0] = 0;
+    e.seg_tile_begin[1] = n_tiles;
+  } else {
+    e.n_seg = g.n_seg;
+    for (int s = 0; s < g.n_seg; ++s) {
+      e.seg_tile_begin[s] = n_tiles;
+      n_tiles += g.seg_rows[s] / kTileN;
+    }
+    e.seg_tile_begin[g.n_seg] = n_tiles;
+  }
+  if (g.M <= 0 || n_tiles <= 0) return DFLASH_OK;
+  const double es_ = (double)esize(ctx);
+  const double n_out = g.paired ? (double)g.seg_rows[0] : (double)n_tiles * kTileN;
+  const double w_rows = (double)n_tiles * kTileN;
+  double out_bytes = 0;
+  switch (e.kind) {
+    case EPI_RESID: out_bytes = 2.0 * g.M * n_out * 4; break;
+    case EPI_ARGMAX: out_bytes = (double)g.M * 8; break;
+    default: out_bytes = (double)g.M * n_out * es_; break;
+  }
+  ProfScope prof(ctx, (!ctx->bf16 || ctx->force_simt) ? PK_GEMM_SIMT : PK_GEMM_TC, st,
+                 w_rows * g.K * es_ + (double)g.M * g.K * es_ + out_bytes, 2.0 * g.M * w_rows * g.K);
+
+  if (!ctx->bf16 || ctx->force_simt) {
+    GemmSimtParams p{};
+    for (int s = 0; s < g.n_seg; ++s) p.w[s] = g.w[s];
+    p.paired = g.paired ? 1 : 0;
+    p.x = g.x;
+    p.ldx = g.ldx;
+    p.M = g.M;
+    p.K = g.K;
+    p.w_bf16 = ctx->bf16 ? 1 : 0;
+    p.x_bf16 = ctx->bf16 ? 1 : 0;
+    p.epi = e;
+    launch_gemm_simt(p, n_tiles, st);
+    return cuda_status(cudaGetLastError(), "gemm_simt launch");
+  }
+
+  GemmTcParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.epi = e;
+  p.paired = g.paired ? 1 : 0;
+  p.M = g.M;
+  p.m_tile = std::min(256, (g.M + 15) / 16 * 16);
+  p.m_blocks = (g.M + p.m_tile - 1) / p.m_tile;
+  p.tmem_cols = std::max(32, pow2_at_least(p.m_tile));
+  p.num_kb = g.K / 64;
+  p.n_tiles = n_tiles;
+  p.n_total = n_tiles * kTileN;
+  const int units = n_tiles * p.m_blocks;
+  const int per_sm = p.m_tile <= 64 ? 2 : 1;
+  const int target = ctx->num_sms * per_sm;
+  int splits = std::max(1, (target + units - 1) / units);
+  splits = std::min(splits, std::max(1, p.num_kb / 4));
+  while (splits > 1 && (size_t)splits * g.M * p.n_total > kPartialFloats) --splits;
+  const int kbps = (p.num_kb + splits - 1) / splits;
+  p.kb_per_split = kbps;
+  p.splits = (p.num_kb + kbps - 1) / kbps;
+  const size_t budget = per_sm == 2 ? 110 * 1024 : 220 * 1024;
+  const int sb = kTileN * 64 * 2 + p.m_tile * 128;
+  p.stages = (int)std::min<size_t>(8, (budget - 1024) / sb);
+  if (p.stages < 2) return DFLASH_ERR_UNSUPPORTED;
+  p.partials = ctx->partials;
+  p.counters = ctx->counters + (size_t)g.site * kCountersPerSite;
+  if (units > kCountersPerSite) return DFLASH_ERR_UNSUPPORTED;
+  p.use_pdl = ctx->use_pdl ? 1 : 0;
+  const int box_w = g.paired ? kTileN / 2 : kTileN;
+  const int nmaps = g.paired ? 2 : g.n_seg;
+  for (int s = 0; s < nmaps; ++s)
+    if (!get_map(ctx, g.w[s], g.seg_rows[s], g.K, g.K, box_w, &p.wmap[s])) return DFLASH_ERR_CUDA;
+  if (!get_map(ctx, g.x, g.M, g.K, g.ldx, p.m_tile, &p.xmap)) return DFLASH_ERR_CUDA;
+  return cuda_status(launch_gemm_tc(p, st), "gemm_tc launch");
+}
+
+#define DFL_CHECK(call)                       \
+  do {                                        \
+    dflash_status s_ = (call);                \
+    if (s_ != DFLASH_OK) return s_;           \
+  } while (0)
+
+}  // namespace
+
+extern "C" const char* dflash_status_string(dflash_status s) {
+  switch (s) {
+    case DFLASH_OK: return "ok";
+    case DFLASH_ERR_ARG: return "invalid argument";
+    case DFLASH_ERR_CUDA: return "CUDA call failed";
+    case DFLASH_ERR_OOM: return "out of device memory";
+    case DFLASH_ERR_TIMEOUT: return "device wait timed out";
+    case DFLASH_ERR_DEVICE: return "out-of-range id, page or position on the device";
+    case DFLASH_ERR_UNSUPPORTED: return "unsupported shape";
+  }
+  return "unknown status";
+}
+
+extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, dflash_ctx** out) {
+  if (!cfg || !w || !out) return DFLASH_ERR_ARG;
+  *out = nullptr;
+  const dflash_config& c = *cfg;
+  if (c.hidden <= 0 || c.n_layers < 0 || c.n_q_heads <= 0 || c.n_kv_heads <= 0 || c.head_dim <= 0 ||
+      c.intermediate <= 0 || c.vocab <= 1 || c.n_feat_layers <= 0 || c.target_hidden <= 0 || c.max_block <= 0 ||
+      c.max_batch <= 0 || c.max_inject_rows < 0 || c.page_size <= 0 || !(c.rope_theta > 0.f) || !(c.rms_eps >= 0.f))
+    return DFLASH_ERR_ARG;
+  if (c.mask_token_id < 0 || c.mask_token_id >= c.vocab) return DFLASH_ERR_ARG;
+  if (c.n_q_heads % c.n_kv_heads) return DFLASH_ERR_ARG;
+  if (c.dtype != DFLASH_F32 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
+  if (!w->fc || !w->embed || !w->lm_head || !w->final_norm) return DFLASH_ERR_ARG;
+  if (c.n_layers > 0 && (!w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo || !w->mlp_norm || !w->wgate ||
+                         !w->wup || !w->wdown))
+    return DFLASH_ERR_ARG;
+  // shape support: 128-row weight tiles aligned to segment starts, paired 64-row gate/up tiles
+  const int F = c.n_feat_layers * c.target_hidden;
+  const int kalign = c.dtype == DFLASH_BF16 ? 64 : 32;
+  if (c.head_dim != 64 && c.head_dim != 128) return DFLASH_ERR_UNSUPPORTED;
+  if (c.hidden % 128 || q_dim(c) % 128 || kv_dim(c) % 128 || c.intermediate % 64 || c.vocab % 128)
+    return DFLASH_ERR_UNSUPPORTED;
+  if (c.hidden % kalign || q_dim(c) % kalign || c.intermediate % kalign || F % kalign) return DFLASH_ERR_UNSUPPORTED;
+  if ((c.n_q_heads / c.n_kv_heads) * c.max_block > 128) return DFLASH_ERR_UNSUPPORTED;
+
+  dflash_ctx* ctx = new dflash_ctx();
+  ctx->cfg = c;
+  ctx->bf16 = c.dtype == DFLASH_BF16;
+  const char* env = std::getenv("DFLASH_FORCE_SIMT");
+  ctx->force_simt = env && env[0] == '1';
+  env = std::getenv("DFLASH_PDL");
+  ctx->use_pdl = env && env[0] == '1';
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  ctx->fc = w->fc;
+  ctx->embed = w->embed;
+  ctx->lm_head = w->lm_head;
+  ctx->final_norm = w->final_norm;
+  for (int l = 0; l < c.n_layers; ++l) {
+    if (!w->attn_norm[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->mlp_norm[l] || !w->wgate[l] ||
+        !w->wup[l] || !w->wdown[l]) {
+      delete ctx;
+      return DFLASH_ERR_ARG;
+    }
+    ctx->attn_norm.push_back(w->attn_norm[l]);
+    ctx->mlp_norm.push_back(w->mlp_norm[l]);
+    ctx->wq.push_back(w->wq[l]);
+    ctx->wk.push_back(w->wk[l]);
+    ctx->wv.push_back(w->wv[l]);
+    ctx->wo.push_back(w->wo[l]);
+    ctx->wg.push_back(w->wgate[l]);
+    ctx->wu.push_back(w->wup[l]);
+    ctx->wd.push_back(w->wdown[l]);
+  }
+
+  cudaDriverEntryPointQueryResult qres;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
+      qres != cudaDriverEntryPointSuccess || !fn) {
+    delete ctx;
+    return DFLASH_ERR_CUDA;
+  }
+  ctx->encode = reinterpret_cast<EncodeTiledFn>(fn);
+
+  // workspace layout
+  const size_t R = (size_t)c.max_batch * c.max_block;
+  const size_t Rin = std::max(1, c.max_inject_rows);
+  const size_t es = esize(ctx);
+  const int g = c.n_q_heads / c.n_kv_heads;
+  const size_t nr = (size_t)g * c.max_block;
+  ctx->att_rows = ((size_t)kAttnTargetCtas + (size_t)c.max_batch * c.n_kv_heads + 8) * nr;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t o_x = take(R * c.hidden * 4);
+  const size_t o_h = take(R * c.hidden * es);
+  const size_t o_q = take(R * q_dim(c) * es);
+  const size_t o_kb = take(R * kv_dim(c) * es);
+  const size_t o_vb = take(R * kv_dim(c) * es);
+  const size_t o_ao = take(R * q_dim(c) * es);
+  const size_t o_act = take(R * c.intermediate * es);
+  const size_t o_c = take(Rin * c.hidden * es);
+  const size_t o_part = take(ctx->bf16 ? kPartialFloats * 4 : 256);
+  const size_t o_ctr = take((size_t)kNumSites * kCountersPerSite * 4);
+  const size_t o_keys = take(R * 8);
+  const size_t o_atto = take(ctx->att_rows * c.head_dim * 4);
+  const size_t o_attm = take(ctx->att_rows * 4);
+  const size_t o_attl = take(ctx->att_rows * 4);
+  const size_t o_st = take(256);
+  ctx->ws_bytes = off;
+  if (cudaMalloc(&ctx->ws, off) != cudaSuccess) {
+    cudaGetLastError();
+    delete ctx;
+    return DFLASH_ERR_OOM;
+  }
+  if (cudaMemset(ctx->ws, 0, off) != cudaSuccess) {
+    cudaFree(ctx->ws);
+    delete ctx;
+    return DFLASH_ERR_CUDA;
+  }
+  char* b = ctx->ws;
+  ctx->x = (float*)(b + o_x);
+  ctx->h = b + o_h;
+  ctx->q = b + o_q;
+  ctx->kb = b + o_kb;
+  ctx->vb = b + o_vb;
+  ctx->ao = b + o_ao;
+  ctx->act = b + o_act;
+  ctx->c = b + o_c;
+  ctx->partials = (float*)(b + o_part);
+  ctx->counters = (int*)(b + o_ctr);
+  ctx->keys = (unsigned long long*)(b + o_keys);
+  ctx->att_o = (float*)(b + o_atto);
+  ctx->att_m = (float*)(b + o_attm);
+  ctx->att_l = (float*)(b + o_attl);
+  ctx->status = (int*)(b + o_st);
+  *out = ctx;
+  return DFLASH_OK;
+}
+
+extern "C" void dflash_destroy(dflash_ctx* ctx) {
+  if (!ctx) return;
+  cudaDeviceSynchronize();
+  cudaFree(ctx->ws);
+  delete ctx;
+}
+
+extern "C" dflash_status dflash_profile_enable(dflash_ctx* ctx, int enable) {
+  if (!ctx) return DFLASH_ERR_ARG;
+  ctx->prof = enable != 0;
+  return DFLASH_OK;
+}
+
+extern "C" int dflash_profile_read(dflash_ctx* ctx, dflash_profile_entry* out, int max_entries) {
+  if (!ctx || (!out && max_entries > 0)) return -(int)DFLASH_ERR_ARG;
+  dflash_profile_entry agg[PK_COUNT];
+  std::memset(agg, 0, sizeof(agg));
+  bool fail = false;
+  for (ProfRec& r : ctx->recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) fail = true;
+    agg[r.kind].launches += 1;
+    agg[r.kind].total_ms += ms;
+    agg[r.kind].bytes += r.bytes;
+    agg[r.kind].flops += r.flops;
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  ctx->recs.clear();
+  if (fail) return -(int)DFLASH_ERR_CUDA;
+  int n = 0;
+  for (int k = 0; k < PK_COUNT; ++k) {
+    if (!agg[k].launches) continue;
+    if (n < max_entries) {
+      out[n] = agg[k];
+      std::strncpy(out[n].name, kProfNames[k], sizeof(out[n].name) - 1);
+    }
+    ++n;
+  }
+  return std::min(n, max_entries);
+}
+
+extern "C" dflash_status dflash_get_error(dflash_ctx* ctx, void* stream) {
+  if (!ctx) return DFLASH_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DFLASH_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ctx->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DFLASH_ERR_CUDA;
+  if (v && cudaMemset(ctx->status, 0, sizeof(int)) != cudaSuccess) return DFLASH_ERR_CUDA;
+  if (v & ST_TIMEOUT) return DFLASH_ERR_TIMEOUT;
+  if (v) return DFLASH_ERR_DEVICE;
+  return DFLASH_OK;
+}
+
+extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, int bs, int max_new,
+                                           const int* d_n_new, const int* d_start_pos, void* const* k_cache,
+                                           void* const* v_cache, const int* d_page_table, int max_pages,
+                                           int num_pages, void* stream) {
+  if (!ctx) return DFLASH_ERR_ARG;
+  const dflash_config& c = ctx->cfg;
+  if (bs <= 0 || bs > c.max_batch || max_new < 0 || (long long)bs * max_new > c.max_inject_rows)
+    return DFLASH_ERR_ARG;
+  if (max_new == 0) return DFLASH_OK;
+  if (!feats || !d_n_new || !d_start_pos || !d_page_table || max_pages <= 0 || num_pages <= 0) return DFLASH_ERR_ARG;
+  if (c.n_layers > 0 && (!k_cache || !v_cache)) return DFLASH_ERR_ARG;
+  for (int l = 0; l < c.n_layers; ++l)
+    if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int M = bs * max_new;
+  const int F = c.n_feat_layers * c.target_hidden;
+
+  GemmSpec fcg;
+  fcg.x = feats;
+  fcg.ldx = F;
+  fcg.M = M;
+  fcg.K = F;
+  fcg.n_seg = 1;
+  fcg.w[0] = ctx->fc;
+  fcg.seg_rows[0] = c.hidden;
+  fcg.site = SITE_FC;
+  fcg.epi.kind = EPI_STORE;
+  fcg.epi.out[0] = ctx->c;
+  fcg.epi.ld_out[0] = c.hidden;
+  fcg.epi.rows_per_req = max_new;
+  DFL_CHECK(run_gemm(ctx, fcg, st));
+
+  // all layers' K and V projections of c, up to kMaxSeg segments per launch
+  const int per_launch = kMaxSeg / 2;
+  for (int l0 = 0, part = 0; l0 < c.n_layers; l0 += per_launch, ++part) {
+    const int nl = std::min(per_launch, c.n_layers - l0);
+    GemmSpec kv;
+    kv.x = ctx->c;
+    kv.ldx = c.hidden;
+    kv.M = M;
+    kv.K = c.hidden;
+    kv.n_seg = 2 * nl;
+    kv.site = SITE_KV + part;
+    EpiParams& e = kv.epi;
+    e.kind = EPI_KV_INJECT;
+    for (int i = 0; i < nl; ++i) {
+      kv.w[2 * i] = ctx->wk[l0 + i];
+      kv.w[2 * i + 1] = ctx->wv[l0 + i];
+      kv.seg_rows[2 * i] = kv.seg_rows[2 * i + 1] = kv_dim(c);
+      e.out[2 * i] = k_cache[l0 + i];
+      e.out[2 * i + 1] = v_cache[l0 + i];
+      e.rope_mask |= 1u << (2 * i);
+    }
+    e.head_dim = c.head_dim;
+    e.log2_theta = std::log2((double)c.rope_theta);
+    e.rows_per_req = max_new;
+    e.pos_base = d_start_pos;
+    e.row_count = d_n_new;
+    e.page_table = d_page_table;
+    e.max_pages = max_pages;
+    e.num_pages = num_pages;
+    e.page_size = c.page_size;
+    e.n_kv = c.n_kv_heads;
+    DFL_CHECK(run_gemm(ctx, kv, st));
+  }
+  return DFLASH_OK;
+}
+
+extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_len, int bs,
+                                            int B, const void* const* k_cache, const void* const* v_cache,
+                                            const int* d_page_table, int max_pages, int num_pages, int max_ctx,
+                                            int* d_draft, float* d_hidden_out, void* stream) {
+  if (!ctx) return DFLASH_ERR_ARG;
+  const dflash_config& c = ctx->cfg;
+  if (bs <= 0 || bs > c.max_batch || B <= 0 || B > c.max_block || max_ctx < 0) return DFLASH_ERR_ARG;
+  if (!d_anchor || !d_ctx_len || (B > 1 && !d_draft)) return DFLASH_ERR_ARG;
+  if (c.n_layers > 0 && (!k_cache || !v_cache)) return DFLASH_ERR_ARG;
+  for (int l = 0; l < c.n_layers; ++l)
+    if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_ARG;
+  if (max_ctx > 0 && (!d_page_table || max_pages <= 0 || num_pages <= 0)) return DFLASH_ERR_ARG;
+  if (max_ctx > (long long)max_pages * c.page_size) return DFLASH_ERR_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int R = bs * B;
+  const int H = c.hidden, QD = q_dim(c), KVD = kv_dim(c);
+  const int hb = ctx->bf16 ? 1 : 0;
+  const size_t layer_stride = (size_t)R * H;
+
+  const double es = (double)esize(ctx);
+  {
+    ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
+    launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, B, R, c.vocab, H,
+                      c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps, ctx->x, ctx->h, hb,
+                      ctx->status, st);
+  }
+  if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+  const double norm_bytes = (double)R * H * (4 + es);
+
+  // attention split plan
+  const int g = c.n_q_heads / c.n_kv_heads;
+  const int T_max = max_ctx + B;
+  int n_splits = std::max(1, (kAttnTargetCtas + bs * c.n_kv_heads - 1) / (bs * c.n_kv_heads));
+  n_splits = std::min(n_splits, (T_max + 31) / 32);
+  int kps = (T_max + n_splits - 1) / n_splits;
+  kps = (kps + 31) / 32 * 32;
+  n_splits = (T_max + kps - 1) / kps;
+  if ((size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows) return DFLASH_ERR_UNSUPPORTED;
+
+  for (int l = 0; l < c.n_layers; ++l) {
+    const int site = SITE_LAYER0 + 4 * l;
+    GemmSpec qkv;
+    qkv.x = ctx->h;
+    qkv.ldx = H;
+    qkv.M = R;
+    qkv.K = H;
+    qkv.n_seg = 3;
+    qkv.w[0] = ctx->wq[l];
+    qkv.w[1] = ctx->wk[l];
+    qkv.w[2] = ctx->wv[l];
+    qkv.seg_rows[0] = QD;
+    qkv.seg_rows[1] = KVD;
+    qkv.seg_rows[2] = KVD;
+    qkv.site = site;
+    qkv.epi.kind = EPI_QKV;
+    qkv.epi.out[0] = ctx->q;
+    qkv.epi.out[1] = ctx->kb;
+    qkv.epi.out[2] = ctx->vb;
+    qkv.epi.ld_out[0] = QD;
+    qkv.epi.ld_out[1] = KVD;
+    qkv.epi.ld_out[2] = KVD;
+    qkv.epi.rope_mask = 3u;
+    qkv.epi.head_dim = c.head_dim;
+    qkv.epi.log2_theta = std::log2((double)c.rope_theta);
+    qkv.epi.rows_per_req = B;
+    qkv.epi.pos_base = d_ctx_len;
+    DFL_CHECK(run_gemm(ctx, qkv, st));
+
+    AttnParams ap{};
+    ap.q = ctx->q;
+    ap.kblk = ctx->kb;
+    ap.vblk = ctx->vb;
+    ap.kc = k_cache[l];
+    ap.vc = v_cache[l];
+    ap.ctx_len = d_ctx_len;
+    ap.page_table = d_page_table;
+    ap.max_pages = max_pages;
+    ap.num_pages = num_pages;
+    ap.page_size = c.page_size;
+    ap.bs = bs;
+    ap.B = B;
+    ap.n_q = c.n_q_heads;
+    ap.n_kv = c.n_kv_heads;
+    ap.d = c.head_dim;
+    ap.g = g;
+    ap.kps = kps;
+    ap.n_splits = n_splits;
+    ap.max_ctx = max_ctx;
+    ap.scale = (float)(1.0 / std::sqrt((double)c.head_dim));
+    ap.part_o = ctx->att_o;
+    ap.part_m = ctx->att_m;
+    ap.part_l = ctx->att_l;
+    ap.status = ctx->status;
+    {
+      // context K/V of every request (upper bound max_ctx), block q/k/v, output
+      const double kvb = (double)bs * max_ctx * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;
+      const double fl = 4.0 * bs * B * (double)(max_ctx + B) * QD;
+      ProfScope prof(ctx, PK_ATTN, st, kvb, fl);
+      DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, hb, hb, st), "attention launch"));
+    }
+
+    GemmSpec o;
+    o.x = ctx->ao;
+    o.ldx = QD;
+    o.M = R;
+    o.K = QD;
+    o.n_seg = 1;
+    o.w[0] = ctx->wo[l];
+    o.seg_rows[0] = H;
+    o.site = site + 1;
+    o.epi.kind = EPI_RESID;
+    o.epi.x = ctx->x;
+    o.epi.ldx = H;
+    DFL_CHECK(run_gemm(ctx, o, st));
+
+    {
+      ProfScope prof(ctx, PK_RMSNORM, st, norm_bytes, 0);
+      launch_rmsnorm(ctx->x, R, H, ctx->mlp_norm[l], c.rms_eps, ctx->h, hb, nullptr, st);
+    }
+
+    GemmSpec gu;
+    gu.x = ctx->h;
+    gu.ldx = H;
+    gu.M = R;
+    gu.K = H;
+    gu.n_seg = 2;
+    gu.paired = true;
+    gu.w[0] = ctx->wg[l];
+    gu.w[1] = ctx->wu[l];
+    gu.seg_rows[0] = gu.seg_rows[1] = c.intermediate;
+    gu.site = site + 2;
+    gu.epi.kind = EPI_SWIGLU;
+    gu.epi.out[0] = ctx->act;
+    gu.epi.ld_out[0] = c.intermediate;
+    DFL_CHECK(run_gemm(ctx, gu, st));
+
+    GemmSpec dn;
+    dn.x = ctx->act;
+    dn.ldx = c.intermediate;
+    dn.M = R;
+    dn.K = c.intermediate;
+    dn.n_seg = 1;
+    dn.w[0] = ctx->wd[l];
+    dn.seg_rows[0] = H;
+    dn.site = site + 3;
+    dn.epi.kind = EPI_RESID;
+    dn.epi.x = ctx->x;
+    dn.epi.ldx = H;
+    DFL_CHECK(run_gemm(ctx, dn, st));
+
+    if (d_hidden_out) {
+      ProfScope prof(ctx, PK_COPY, st, (double)layer_stride * 8, 0);
+      if (cudaMemcpyAsync(d_hidden_out + l * layer_stride, ctx->x, layer_stride * 4, cudaMemcpyDeviceToDevice,
+                          st) != cudaSuccess)
+        return DFLASH_ERR_CUDA;
+    }
+    const bool last = l + 1 == c.n_layers;
+    {
+      ProfScope prof(ctx, PK_RMSNORM, st, norm_bytes, 0);
+      launch_rmsnorm(ctx->x, R, H, last ? ctx->final_norm : ctx->attn_norm[l + 1], c.rms_eps, ctx->h, hb,
+                     last && d_hidden_out ? d_hidden_out + (size_t)c.n_layers * layer_stride : nullptr, st);
+    }
+  }
+  if (c.n_layers == 0 && d_hidden_out)
+    launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, ctx->h, hb, d_hidden_out, st);
+  if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+
+  GemmSpec lm;
+  lm.x = ctx->h;
+  lm.ldx = H;
+  lm.M = R;
+  lm.K = H;
+  lm.n_seg = 1;
+  lm.w[0] = ctx->lm_head;
+  lm.seg_rows[0] = c.vocab;
+  lm.site = SITE_LM;
+  lm.epi.kind = EPI_ARGMAX;
+  lm.epi.keys = ctx->keys;
+  DFL_CHECK(run_gemm(ctx, lm, st));
+  {
+    ProfScope prof(ctx, PK_ARGMAX, st, (double)R * 8 * 2 + (double)bs * (B - 1) * 4, 0);
+    launch_argmax_finalize(ctx->keys, bs, B, d_draft, st);
+  }
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}

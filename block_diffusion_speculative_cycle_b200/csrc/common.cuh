@@ -1,0 +1,100 @@
+// Shared device helpers for the DFlash draft-cycle kernels (sm_100a).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dfl {
+
+// ---------------------------------------------------------------- status bits
+// Kernels record problems here and skip the offending element; they never trap.
+enum : int {
+  ST_BAD_TOKEN = 1,     // a token id outside [0, V)
+  ST_BAD_PAGE = 2,      // a page id outside [0, num_pages) or a page slot beyond max_pages
+  ST_TIMEOUT = 4,       // a bounded wait gave up
+  ST_BAD_CTX = 8,       // a context length outside [0, max_ctx]
+};
+
+__device__ __forceinline__ void flag_error(int* status, int bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// ---------------------------------------------------------------- element conversion
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// ---------------------------------------------------------------- argmax keys
+// A (value, index) pair packed so that the unsigned 64-bit maximum is the
+// largest value and, among equal values, the lowest index. NaN ranks below
+// every number (-inf included) and -0.0 equals +0.0. atomicMax on these keys is
+// order-independent, hence deterministic.
+__device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
+  unsigned int u;
+  if (v != v) {
+    u = 0u;
+  } else {
+    if (v == 0.0f) v = 0.0f;
+    unsigned int b = __float_as_uint(v);
+    u = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  }
+  return ((unsigned long long)u << 32) | (unsigned long long)(~(unsigned int)idx);
+}
+__device__ __forceinline__ int argmax_key_index(unsigned long long key) {
+  return (int)(~(unsigned int)(key & 0xffffffffull));
+}
+
+__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
+  unsigned int lo = (unsigned int)v, hi = (unsigned int)(v >> 32);
+  lo = __shfl_xor_sync(0xffffffffu, lo, m);
+  hi = __shfl_xor_sync(0xffffffffu, hi, m);
+  return ((unsigned long long)hi << 32) | lo;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) {
+    unsigned long long o = shfl_xor_u64(v, m);
+    v = o > v ? o : v;
+  }
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
+  return v;
+}
+
+// ---------------------------------------------------------------- time
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Every spin in these kernels gives up after this long and flags ST_TIMEOUT.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// ---------------------------------------------------------------- RoPE
+// Rotate-half RoPE factor for pair index i (0 <= i < d/2) at position pos:
+// angle = pos * theta^(-2i/d), evaluated in double so that long contexts keep
+// full fp32 accuracy in cos/sin.
+__device__ __forceinline__ void rope_cos_sin(int pos, int i, int d, double log2_theta, float* c, float* s) {
+  double inv_freq = exp2(-2.0 * (double)i / (double)d * log2_theta);
+  double ang = (double)pos * inv_freq;
+  double sd, cd;
+  sincos(ang, &sd, &cd);
+  *c = (float)cd;
+  *s = (float)sd;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+}  // namespace dfl

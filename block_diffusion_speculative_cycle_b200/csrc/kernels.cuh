@@ -1,0 +1,41 @@
+// Launch interfaces of the non-GEMM kernels of the draft cycle.
+#pragma once
+
+#include "common.cuh"
+
+namespace dfl {
+
+struct AttnParams {
+  const void* q;              // [R, n_q*d] block queries (RoPE applied)
+  const void* kblk;           // [R, n_kv*d] block keys (RoPE applied)
+  const void* vblk;           // [R, n_kv*d] block values
+  const void* kc;             // cache pool [num_pages, n_kv, page_size, d]
+  const void* vc;
+  const int* ctx_len;         // [bs]
+  const int* page_table;      // [bs, max_pages]
+  int max_pages, num_pages, page_size;
+  int bs, B, n_q, n_kv, d, g;
+  int kps;                    // keys per split
+  int n_splits;
+  int max_ctx;
+  float scale;                // 1/sqrt(d)
+  float* part_o;              // [bs, n_kv, n_splits, g*B, d]
+  float* part_m;              // [bs, n_kv, n_splits, g*B]
+  float* part_l;
+  int* status;
+};
+
+// Split-KV attention partials, then the log-sum-exp merge into out [R, n_q*d].
+cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st);
+
+// x[m] = E[token(m)] (token = anchor for block index 0, mask id otherwise), h[m] = RMSNorm(x[m]) * gain.
+void launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
+                       int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
+                       cudaStream_t st);
+// h[m] = RMSNorm(x[m]) * gain; optional fp32 copy of h into y.
+void launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
+                    cudaStream_t st);
+// draft[b, i-1] = index(keys[b*B + i]) for i >= 1; every key reset to 0.
+void launch_argmax_finalize(unsigned long long* keys, int bs, int B, int* draft, cudaStream_t st);
+
+}  // namespace dfl

@@ -1,0 +1,135 @@
+// Greedy verify of a drafted block against the target's block logits.
+//
+// Grid (chunk, row j, request b): each CTA streams one chunk of one logits row
+// with 16-byte loads, reduces a packed (value, index) key and folds it into
+// keys[b, j] with atomicMax (order-independent, so bit-reproducible). The last
+// CTA of a request (atomic ticket) walks the B rows: a = leading matches of
+// draft[i-1] against argmax row i-1, next = argmax row a; it then zeroes the
+// request's keys and ticket so the workspace is ready for the next call.
+#include "../../include/dflash.h"
+#include "common.cuh"
+
+namespace dfl {
+
+constexpr int kVerifyThreads = 256;
+constexpr int kVerifyChunk = 8192;   // logits per CTA
+
+template <typename T>
+__device__ __forceinline__ unsigned long long chunk_best(const T* row, int v0, int v1);
+
+template <>
+__device__ __forceinline__ unsigned long long chunk_best<__nv_bfloat16>(const __nv_bfloat16* row, int v0, int v1) {
+  unsigned long long best = 0ull;
+  // 8 bf16 per 16-byte load when the chunk start is 16-byte aligned
+  const bool vec = ((reinterpret_cast<uintptr_t>(row + v0) & 15) == 0);
+  int v = v0;
+  if (vec) {
+    const int nvec = (v1 - v0) / 8;
+    const uint4* p = reinterpret_cast<const uint4*>(row + v0);
+    for (int e = threadIdx.x; e < nvec; e += blockDim.x) {
+      const uint4 u = __ldcs(p + e);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xffff0000u);
+        const int idx = v0 + e * 8 + 2 * k;
+        unsigned long long a = argmax_key(lo, idx), b = argmax_key(hi, idx + 1);
+        a = a > b ? a : b;
+        best = a > best ? a : best;
+      }
+    }
+    v = v0 + nvec * 8;
+  }
+  for (int e = v + threadIdx.x; e < v1; e += blockDim.x) {
+    const unsigned long long a = argmax_key(__bfloat162float(row[e]), e);
+    best = a > best ? a : best;
+  }
+  return best;
+}
+
+template <>
+__device__ __forceinline__ unsigned long long chunk_best<float>(const float* row, int v0, int v1) {
+  unsigned long long best = 0ull;
+  const bool vec = ((reinterpret_cast<uintptr_t>(row + v0) & 15) == 0);
+  int v = v0;
+  if (vec) {
+    const int nvec = (v1 - v0) / 4;
+    const float4* p = reinterpret_cast<const float4*>(row + v0);
+    for (int e = threadIdx.x; e < nvec; e += blockDim.x) {
+      const float4 f = __ldcs(p + e);
+      const float w[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const unsigned long long a = argmax_key(w[k], v0 + e * 4 + k);
+        best = a > best ? a : best;
+      }
+    }
+    v = v0 + nvec * 4;
+  }
+  for (int e = v + threadIdx.x; e < v1; e += blockDim.x) {
+    const unsigned long long a = argmax_key(row[e], e);
+    best = a > best ? a : best;
+  }
+  return best;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kVerifyThreads) verify_kernel(const T* logits, const int* draft, int B, int V,
+                                                                 unsigned long long* keys, int* tickets,
+                                                                 int* accepted, int* next_token) {
+  __shared__ unsigned long long red[kVerifyThreads / 32];
+  const int c = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
+  const T* row = logits + ((size_t)b * B + j) * V;
+  const int v0 = c * kVerifyChunk, v1 = min(V, v0 + kVerifyChunk);
+  unsigned long long best = warp_max_u64(chunk_best<T>(row, v0, v1));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kVerifyThreads / 32; ++w) best = red[w] > best ? red[w] : best;
+    atomicMax(keys + (size_t)b * B + j, best);
+    __threadfence();
+    const int total = (int)gridDim.x * B;
+    const int prev = atomicAdd(tickets + b, 1);
+    if (prev == total - 1) {
+      __threadfence();
+      unsigned long long* kb = keys + (size_t)b * B;
+      int a = 0;
+      while (a < B - 1 && draft[(size_t)b * (B - 1) + a] == argmax_key_index(__ldcg(kb + a))) ++a;
+      accepted[b] = a;
+      next_token[b] = argmax_key_index(__ldcg(kb + a));
+      for (int r = 0; r < B; ++r) kb[r] = 0ull;
+      tickets[b] = 0;
+    }
+  }
+}
+
+}  // namespace dfl
+
+extern "C" size_t dflash_verify_workspace_size(int bs, int B) {
+  if (bs <= 0 || B <= 0) return 0;
+  const size_t keys = (size_t)bs * B * sizeof(unsigned long long);
+  return keys + (((size_t)bs * sizeof(int) + 255) / 256) * 256;
+}
+
+extern "C" dflash_status dflash_verify(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft, int bs,
+                                       int B, int V, int* d_accepted, int* d_next_token, void* d_workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (bs <= 0 || B <= 0 || V <= 0 || !d_logits || !d_accepted || !d_next_token || !d_workspace) return DFLASH_ERR_ARG;
+  if (B > 1 && !d_draft) return DFLASH_ERR_ARG;
+  if (logits_dtype != DFLASH_F32 && logits_dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
+  if (workspace_bytes < dflash_verify_workspace_size(bs, B)) return DFLASH_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_workspace) & 7) != 0) return DFLASH_ERR_ARG;
+  if (bs > 65535 || B > 65535) return DFLASH_ERR_UNSUPPORTED;
+  auto* keys = reinterpret_cast<unsigned long long*>(d_workspace);
+  auto* tickets = reinterpret_cast<int*>(reinterpret_cast<char*>(d_workspace) + (size_t)bs * B * 8);
+  const dim3 grid((unsigned)((V + dfl::kVerifyChunk - 1) / dfl::kVerifyChunk), (unsigned)B, (unsigned)bs);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (logits_dtype == DFLASH_BF16)
+    dfl::verify_kernel<__nv_bfloat16><<<grid, dfl::kVerifyThreads, 0, st>>>(
+        (const __nv_bfloat16*)d_logits, d_draft, B, V, keys, tickets, d_accepted, d_next_token);
+  else
+    dfl::verify_kernel<float><<<grid, dfl::kVerifyThreads, 0, st>>>((const float*)d_logits, d_draft, B, V, keys,
+                                                                    tickets, d_accepted, d_next_token);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}

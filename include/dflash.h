@@ -1,0 +1,216 @@
+/*
+ * dflash.h — C ABI of the B200 (sm_100a) DFlash draft-cycle library.
+ *
+ * One draft cycle of block-diffusion speculative decoding has three calls:
+ *
+ *   dflash_inject_ctx   target features -> per-layer injected K/V in the drafter cache
+ *   dflash_draft_block  anchor + cache -> B-1 draft tokens in one non-causal pass
+ *   dflash_verify       target block logits + drafts -> accepted length, next token
+ *
+ * Sources (page title, section):
+ *   [P1] "DFlash — 블록 확산 드래프터로 6배 빨라지는 투기적 디코딩": §1 greedy verify,
+ *        §2 the cycle (anchor, B-1 masks, one drafter pass, one verify pass) and
+ *        KV injection, §6 non-causal in-block attention.
+ *   [P2] "한 번에 초안을 생성하는 DFlash ...": features of uniformly spaced target
+ *        layers, fused by a lightweight projection, injected into every drafter
+ *        layer's Key/Value.
+ *   [P3] "기술 요약: DFlash – 플래시 추측적 디코딩을 위한 블록 확산": §2.2 context feature
+ *        extraction, KV injection into the drafter's KV cache, parallel block
+ *        prediction in one forward pass; §2.3 embedding and LM head shared with
+ *        the target and frozen.
+ *   [P4] "DFlash 소개" (forum post): the spec_generate(target, draft, input_ids,
+ *        num_speculative_tokens, temperature, max_new_tokens) call shape.
+ *
+ * Conventions for every entry point
+ *   - All tensors are caller-owned device memory, row-major, densely packed
+ *     unless a leading dimension is given. The library never frees them.
+ *   - "stream" is a cudaStream_t (NULL = legacy default stream). Every call is
+ *     asynchronous on it and enqueues kernels only: no host synchronisation, no
+ *     allocation, so a whole cycle can be captured in a CUDA graph.
+ *   - Argument errors are detected on the host before any launch and returned
+ *     as DFLASH_ERR_ARG / DFLASH_ERR_UNSUPPORTED; nothing is enqueued then.
+ *   - Errors found by kernels (a token id, page id or position out of range; a
+ *     bounded device wait that gave up) are recorded in a device status word;
+ *     the offending element is skipped, the kernel returns normally, and
+ *     dflash_get_error() reports and clears it. Kernels never trap.
+ *   - Inputs that change from cycle to cycle (anchor, context length, n_new,
+ *     start position) are device pointers, so the host never needs to read
+ *     the previous cycle's result.
+ *   - Weights and features are bf16 or fp32 (dflash_config.dtype); RMSNorm
+ *     gains are always fp32. Accumulation is fp32; the draft argmax is taken on
+ *     fp32 logits, which are never written to memory.
+ */
+#ifndef DFLASH_H
+#define DFLASH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DFLASH_OK = 0,
+  DFLASH_ERR_ARG = 1,          /* invalid argument (host-side check) */
+  DFLASH_ERR_CUDA = 2,         /* a CUDA runtime / driver call failed */
+  DFLASH_ERR_OOM = 3,          /* workspace allocation failed (dflash_create only) */
+  DFLASH_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up */
+  DFLASH_ERR_DEVICE = 5,       /* a kernel met an out-of-range id, page or position */
+  DFLASH_ERR_UNSUPPORTED = 6   /* a shape this build has no kernel for */
+} dflash_status;
+
+typedef enum { DFLASH_F32 = 0, DFLASH_BF16 = 1 } dflash_dtype;
+
+/* Drafter shape. Notation of the pages: B = block size (anchor + B-1 masks). */
+typedef struct {
+  int hidden;          /* H */
+  int n_layers;        /* L (5 for the 8B-class drafters, 8 for the coder drafter) */
+  int n_q_heads;       /* n_q */
+  int n_kv_heads;      /* n_kv; n_q % n_kv == 0, query head j reads kv head j / (n_q/n_kv) */
+  int head_dim;        /* d: 64 or 128 */
+  int intermediate;    /* SwiGLU width I */
+  int vocab;           /* V (shared with the target) */
+  int n_feat_layers;   /* n_f: number of tapped target layers */
+  int target_hidden;   /* H_t: feature width per tapped layer */
+  int mask_token_id;   /* id fed at the B-1 masked positions, 0 <= id < V */
+  int max_block;       /* largest B passed to dflash_draft_block / dflash_verify */
+  int max_batch;       /* largest bs */
+  int max_inject_rows; /* largest bs * max_new passed to dflash_inject_ctx */
+  int page_size;       /* tokens per KV page (64 in the batched workloads) */
+  float rope_theta;    /* rotary base theta; pair (i, i+d/2) turns by pos * theta^(-2i/d) */
+  float rms_eps;       /* RMSNorm epsilon */
+  dflash_dtype dtype;  /* storage type of weights, features and the KV cache */
+} dflash_config;
+
+/* Weights: device pointers, [out_features, in_features] row-major, in
+ * config.dtype (norm gains: fp32 [H]). Per-layer entries are HOST arrays of
+ * n_layers device pointers; the library copies the pointer values at create
+ * time and keeps them (the tensors must outlive the context).
+ *   fc      [H, n_f*H_t]   lightweight projection of the concatenated features
+ *   embed   [V, H]         target-owned token embedding (shared, frozen)
+ *   lm_head [V, H]         target-owned LM head (may equal embed)
+ *   wq [n_q*d, H], wk/wv [n_kv*d, H], wo [H, n_q*d],
+ *   wgate/wup [I, H], wdown [H, I]                                          */
+typedef struct {
+  const void* fc;
+  const void* embed;
+  const void* lm_head;
+  const float* final_norm;
+  const float* const* attn_norm;
+  const void* const* wq;
+  const void* const* wk;
+  const void* const* wv;
+  const void* const* wo;
+  const float* const* mlp_norm;
+  const void* const* wgate;
+  const void* const* wup;
+  const void* const* wdown;
+} dflash_weights;
+
+typedef struct dflash_ctx dflash_ctx;
+
+/* Create a drafter context. Validates the shape, encodes the weights' TMA
+ * descriptors and allocates the library's own workspace (activations, split-K
+ * partials, argmax keys, a device status word) on the current device.
+ * Returns DFLASH_ERR_UNSUPPORTED for shapes without a kernel (bf16 needs H,
+ * n_q*d, n_kv*d, I, V multiples of 128 and n_f*H_t a multiple of 64).
+ * On success *out owns the context; release it with dflash_destroy. */
+dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, dflash_ctx** out);
+
+/* Free the context and its workspace (synchronises the device first). NULL is a no-op. */
+void dflash_destroy(dflash_ctx* ctx);
+
+/* KV injection ([P3] §2.2, [P2], [P1] §2): c = F · W_fcᵀ, then for every layer l
+ * K_l = RoPE(c · Wk_lᵀ) at the row's absolute position and V_l = c · Wv_lᵀ,
+ * written into that layer's cache pages. No norm precedes Wk/Wv here.
+ *
+ *   feats       [bs, max_new, n_f*H_t] (dtype): features of the tapped target
+ *               layers, concatenated shallow -> deep; rows >= n_new[r] are ignored
+ *   d_n_new     [bs] int32 (device): rows to inject per request, 0..max_new
+ *   d_start_pos [bs] int32 (device): absolute position of request r's first row
+ *   k_cache, v_cache: HOST arrays [n_layers] of device pointers to page pools
+ *               [num_pages, n_kv, page_size, d] (dtype)
+ *   d_page_table [bs, max_pages] int32 (device): page of token block p of request r
+ * A position whose page slot is beyond max_pages, or whose page id is outside
+ * [0, num_pages), is skipped and flagged (DFLASH_ERR_DEVICE). */
+dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, int bs, int max_new,
+                                const int* d_n_new, const int* d_start_pos,
+                                void* const* k_cache, void* const* v_cache,
+                                const int* d_page_table, int max_pages, int num_pages,
+                                void* stream);
+
+/* One drafter pass over the block ([P1] §2 steps 1-3, §6; [P3] §2.2):
+ * rows (r, i), i < B, hold E[anchor_r] (i = 0) or E[mask_token_id] at position
+ * ctx_len[r] + i. Every layer: RMSNorm -> q,k,v (RoPE on q,k) -> attention of
+ * each block query over the request's injected context K/V (positions
+ * 0..ctx_len[r]-1) and all B block keys, no mask -> Wo + residual; RMSNorm ->
+ * SwiGLU MLP + residual. Then the final RMSNorm, the shared LM head and a
+ * greedy argmax (lowest id on ties) per masked row, fused: logits are never
+ * stored. The block's own K/V are not written to the cache.
+ *
+ *   d_anchor  [bs] int32 (device): last accepted token per request
+ *   d_ctx_len [bs] int32 (device): injected context length P_r, 0 <= P_r <= max_ctx
+ *   max_ctx   host upper bound on every P_r (sizes the attention split grid)
+ *   d_draft   [bs, B-1] int32 (device, out): d_1..d_{B-1}
+ *   d_hidden_out: NULL, or [L+1, bs, B, H] fp32 (device, out): the residual
+ *               stream after each layer, then the final normed rows (for parity
+ *               checks; costs extra writes). */
+dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_len, int bs, int B,
+                                 const void* const* k_cache, const void* const* v_cache,
+                                 const int* d_page_table, int max_pages, int num_pages, int max_ctx,
+                                 int* d_draft, float* d_hidden_out, void* stream);
+
+/* Bytes of scratch dflash_verify needs for (bs, B). */
+size_t dflash_verify_workspace_size(int bs, int B);
+
+/* Greedy verify ([P1] §1, §2 step 4): g_j = argmax_v logits[r, j, v] (lowest
+ * index on ties, NaN below every number, -0 == +0, compared in fp32);
+ * a_r = number of leading i >= 1 with draft[r, i-1] == g_{i-1};
+ * next_r = g_{a_r} (the correction, or the bonus token when a_r = B-1).
+ * The committed tokens are draft[r, 0..a_r-1] followed by next_r.
+ *
+ *   d_logits    [bs, B, V] in logits_dtype (device)
+ *   d_draft     [bs, B-1] int32 (device)
+ *   d_accepted, d_next_token [bs] int32 (device, out)
+ *   d_workspace at least dflash_verify_workspace_size(bs, B) bytes of device
+ *               memory, zero-filled before its first use; every call leaves
+ *               it zero-filled again. Calls that share a workspace must not
+ *               overlap on the GPU.
+ * Independent of any drafter context. Results are bit-exact given the logits. */
+dflash_status dflash_verify(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft,
+                            int bs, int B, int V, int* d_accepted, int* d_next_token,
+                            void* d_workspace, size_t workspace_bytes, void* stream);
+
+/* Per-kernel timing, an instrumentation hook with no counterpart on the pages.
+ * While enabled, every kernel this context launches is bracketed by a pair of
+ * CUDA events on its stream, tagged with the launch's algorithmic bytes (each
+ * weight, activation and output element counted once) and flops. Meant for
+ * eager (not graph-captured) profiling passes: it adds event records between
+ * launches. dflash_profile_read synchronises, aggregates per kernel kind and
+ * clears the records. */
+typedef struct {
+  char name[32];      /* kernel kind: "gemm_tc", "gemm_simt", "attention", "rmsnorm", ... */
+  int launches;
+  double total_ms;    /* summed event-to-event durations */
+  double bytes;       /* algorithmic bytes summed over the launches */
+  double flops;       /* algorithmic flops summed over the launches */
+} dflash_profile_entry;
+
+dflash_status dflash_profile_enable(dflash_ctx* ctx, int enable);
+
+/* Fill up to max_entries aggregated entries; returns how many were written
+ * (negative dflash_status on error). Resets the records. */
+int dflash_profile_read(dflash_ctx* ctx, dflash_profile_entry* out, int max_entries);
+
+/* Synchronise `stream`, read and clear the context's device status word.
+ * Returns DFLASH_ERR_TIMEOUT, DFLASH_ERR_DEVICE or DFLASH_OK. */
+dflash_status dflash_get_error(dflash_ctx* ctx, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* dflash_status_string(dflash_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DFLASH_H */

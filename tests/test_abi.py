@@ -1,0 +1,54 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds, loads and
+exports every entry point include/dflash.h declares, and the binding declares
+the same names."""
+import os
+import re
+
+import pytest
+
+from block_diffusion_speculative_cycle_b200 import _binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    src = open(os.path.join(ROOT, "include", "dflash.h"), encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dflash_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib_path():
+    return build.build()
+
+
+def test_header_declares_the_cycle_calls():
+    names = declared_entry_points()
+    for n in ("dflash_inject_ctx", "dflash_draft_block", "dflash_verify", "dflash_create", "dflash_destroy"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib_path):
+    exported = _binding.exported_symbols(lib_path)
+    missing = [n for n in declared_entry_points() if n not in exported]
+    assert not missing, missing
+    assert sorted(_binding.EXPORTS) == declared_entry_points()
+
+
+def test_status_strings_and_workspace_size(lib_path):
+    lib = _binding.load_library(lib_path)
+    assert lib.dflash_status_string(0) == b"ok"
+    assert lib.dflash_status_string(5).startswith(b"out-of-range")
+    assert lib.dflash_verify_workspace_size(0, 4) == 0
+    assert lib.dflash_verify_workspace_size(3, 16) >= 3 * 16 * 8 + 3 * 4
+
+
+def test_create_rejects_bad_config_without_touching_the_gpu(lib_path):
+    import ctypes
+    lib = _binding.load_library(lib_path)
+    cfg = _binding.dflash_config()
+    w = _binding.dflash_weights()
+    h = ctypes.c_void_p()
+    assert lib.dflash_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)) == 1   # DFLASH_ERR_ARG
+    assert lib.dflash_create(None, None, ctypes.byref(h)) == 1
+    assert lib.dflash_verify(None, 0, None, 1, 4, 10, None, None, None, 0, None) == 1

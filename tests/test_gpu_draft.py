@@ -1,0 +1,89 @@
+"""dflash_inject_ctx + dflash_draft_block against the oracle on seeded inputs.
+
+Bars: hidden states within max-abs-rel 1e-4 (fp32 drafter) / 2e-2 (bf16
+drafter) per layer and for the final normed rows; draft tokens identical
+wherever the oracle's top-2 logit gap exceeds 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_speculative_cycle_b200 import synth
+from oracle import dflash as O
+from tests.gpu_harness import PagedCache, make_drafter, max_abs_rel, top2_gap
+
+pytestmark = pytest.mark.gpu
+
+SMALL_BF16 = synth.DrafterConfig(name="small-bf16", hidden=512, n_layers=2, n_q_heads=4, n_kv_heads=2,
+                                 head_dim=128, intermediate=1024, vocab=2048, n_feat_layers=3,
+                                 target_hidden=256, rope_theta=1e4, dtype="bf16")
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def run_case(cfg, ctx_lens, B, seed=0, chunks=1, max_new_pad=0, anchors=None, share=True):
+    bs = len(ctx_lens)
+    ctx = torch.tensor(ctx_lens, dtype=torch.int32)
+    w = synth.make_drafter_weights(cfg, seed=seed, share_embed_lm_head=share)
+    page = 64
+    table, num_pages = synth.make_page_table(ctx, page, extra_tokens=B, seed=seed + 1)
+    max_new = max(max(ctx_lens), 1) + max_new_pad
+    feats = synth.make_features(cfg, bs * max_new, seed=seed + 2).reshape(bs, max_new, cfg.feat_dim)
+    if anchors is None:
+        anchors = synth.make_tokens(cfg, bs, seed=seed + 3)
+    drafter, _ = make_drafter(cfg, w, max_block=B, max_batch=bs, max_inject_rows=bs * max_new, page_size=page)
+    cache = PagedCache(cfg, table, num_pages, page)
+
+    # GPU: inject (optionally in several chunks), then one draft pass
+    dev = "cuda"
+    bounds = np.linspace(0, max(ctx_lens), chunks + 1).astype(int)
+    for c0, c1 in zip(bounds[:-1], bounds[1:]):
+        n_new = torch.tensor([max(0, min(P, c1) - c0) for P in ctx_lens], dtype=torch.int32, device=dev)
+        start = torch.full((bs,), int(c0), dtype=torch.int32, device=dev)
+        f = feats[:, c0:c1 + max_new_pad].contiguous().to(dev)
+        drafter.inject(f, bs, f.shape[1], n_new, start, cache.k, cache.v, cache.table, num_pages)
+    draft = torch.zeros((bs, B - 1), dtype=torch.int32, device=dev)
+    hidden = torch.zeros((cfg.n_layers + 1, bs, B, cfg.hidden), dtype=torch.float32, device=dev)
+    drafter.draft(anchors.to(dev), ctx.to(dev), bs, B, cache.k, cache.v, cache.table, num_pages, max(ctx_lens),
+                  draft, hidden)
+    drafter.check()
+    torch.cuda.synchronize()
+    draft, hidden = draft.cpu().numpy(), hidden.cpu().numpy()
+
+    # oracle, request by request, from the same CPU inputs
+    tol = TOL[cfg.dtype]
+    for r in range(bs):
+        P = ctx_lens[r]
+        oc = O.Cache(cfg)
+        if P:
+            oc.write(0, O.inject(cfg, w, feats[r, :P], 0)[1])
+        ref = O.draft_block(cfg, w, int(anchors[r]), oc, B)
+        for l in range(cfg.n_layers + 1):
+            err = max_abs_rel(hidden[l, r], ref["hidden"][l])
+            assert err <= tol, f"request {r} layer {l}: max-abs-rel {err:.3g} > {tol}"
+        if B > 1:
+            gap = top2_gap(ref["logits"])
+            sure = gap > 1e-2
+            np.testing.assert_array_equal(draft[r][sure], ref["draft"][sure])
+    return draft
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_tiny_fp32(B):
+    run_case(synth.TINY, [64], B)
+
+
+def test_tiny_fp32_ragged_batch_chunked_inject():
+    run_case(synth.TINY, [0, 5, 64, 131], 4, seed=3, chunks=3)
+
+
+@pytest.mark.parametrize("ctx_lens,B", [([200], 16), ([0, 77, 300], 10), ([1], 2), ([64, 64], 1)])
+def test_small_bf16(ctx_lens, B):
+    run_case(SMALL_BF16, ctx_lens, B, seed=len(ctx_lens) + B)
+
+
+def test_small_bf16_chunked_inject_and_padding_rows():
+    run_case(SMALL_BF16, [130, 257], 16, seed=11, chunks=4, max_new_pad=3)
+
+
+def test_small_bf16_untied_head_and_many_requests():
+    lens = list(np.random.default_rng(0).integers(0, 400, size=12))
+    run_case(SMALL_BF16, [int(x) for x in lens], 16, seed=5, share=False)
