@@ -21,7 +21,7 @@ _STATUS = {0: "DFLASH_OK", 1: "DFLASH_ERR_ARG", 2: "DFLASH_ERR_CUDA", 3: "DFLASH
            4: "DFLASH_ERR_TIMEOUT", 5: "DFLASH_ERR_DEVICE", 6: "DFLASH_ERR_UNSUPPORTED"}
 
 EXPORTS = ["dflash_create", "dflash_destroy", "dflash_inject_ctx", "dflash_draft_block",
-           "dflash_verify_workspace_size", "dflash_verify", "dflash_profile_enable", "dflash_profile_read",
+           "dflash_verify_workspace_size", "dflash_verify", "dflash_verify_noalloc", "dflash_profile_enable", "dflash_profile_read",
            "dflash_get_error", "dflash_status_string"]
 
 
@@ -79,6 +79,8 @@ def load_library(path: Optional[str] = None):
     lib.dflash_verify_workspace_size.restype = c_size
     lib.dflash_verify.argtypes = [_P, c_int, _P, c_int, c_int, c_int, _P, _P, _P, c_size, _P]
     lib.dflash_verify.restype = c_int
+    lib.dflash_verify_noalloc.argtypes = [_P, c_int, _P, c_int, c_int, c_int, _P, _P, _P]
+    lib.dflash_verify_noalloc.restype = c_int
     lib.dflash_profile_enable.argtypes = [_P, c_int]
     lib.dflash_profile_enable.restype = c_int
     lib.dflash_profile_read.argtypes = [_P, ctypes.POINTER(dflash_profile_entry), c_int]

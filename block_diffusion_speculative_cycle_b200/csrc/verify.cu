@@ -6,6 +6,9 @@
 // CTA of a request (atomic ticket) walks the B rows: a = leading matches of
 // draft[i-1] against argmax row i-1, next = argmax row a; it then zeroes the
 // request's keys and ticket so the workspace is ready for the next call.
+#include <cstdio>
+#include <mutex>
+
 #include "../../include/dflash.h"
 #include "common.cuh"
 
@@ -125,6 +128,66 @@ extern "C" dflash_status dflash_verify(const void* d_logits, dflash_dtype logits
   auto* tickets = reinterpret_cast<int*>(reinterpret_cast<char*>(d_workspace) + (size_t)bs * B * 8);
   const dim3 grid((unsigned)((V + dfl::kVerifyChunk - 1) / dfl::kVerifyChunk), (unsigned)B, (unsigned)bs);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (logits_dtype == DFLASH_BF16)
+    dfl::verify_kernel<__nv_bfloat16><<<grid, dfl::kVerifyThreads, 0, st>>>(
+        (const __nv_bfloat16*)d_logits, d_draft, B, V, keys, tickets, d_accepted, d_next_token);
+  else
+    dfl::verify_kernel<float><<<grid, dfl::kVerifyThreads, 0, st>>>((const float*)d_logits, d_draft, B, V, keys,
+                                                                    tickets, d_accepted, d_next_token);
+  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- no-allocation variant
+// Scratch of dflash_verify_noalloc: keys at offset 0, tickets after the keys.
+// A host-side mention of this name is only a stand-in symbol, not a device
+// address; host code passes the address from cudaGetSymbolAddress instead.
+static __device__ __align__(256) unsigned char g_verify_scratch[DFLASH_VERIFY_NOALLOC_MAX_ROWS * 8 +
+                                                                 DFLASH_VERIFY_NOALLOC_MAX_BATCH * 4];
+
+namespace {
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of g_verify_scratch on the current device, looked up once per device.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_verify_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+extern "C" dflash_status dflash_verify_noalloc(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft,
+                                               int bs, int B, int V, int* d_accepted, int* d_next_token,
+                                               void* stream) {
+  if (bs <= 0 || B <= 0 || V <= 0 || !d_logits || !d_accepted || !d_next_token) return DFLASH_ERR_ARG;
+  if (B > 1 && !d_draft) return DFLASH_ERR_ARG;
+  if (logits_dtype != DFLASH_F32 && logits_dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
+  if (bs > DFLASH_VERIFY_NOALLOC_MAX_BATCH || (long long)bs * B > DFLASH_VERIFY_NOALLOC_MAX_ROWS) {
+    std::fprintf(stderr,
+                 "dflash_verify_noalloc: bs=%d, B=%d exceed the fixed scratch (bs <= %d, bs*B <= %d); "
+                 "use dflash_verify with a caller-provided workspace\n",
+                 bs, B, DFLASH_VERIFY_NOALLOC_MAX_BATCH, DFLASH_VERIFY_NOALLOC_MAX_ROWS);
+    return DFLASH_ERR_ARG;
+  }
+  void* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return DFLASH_ERR_CUDA;
+  auto* keys = reinterpret_cast<unsigned long long*>(scratch);
+  auto* tickets = reinterpret_cast<int*>(reinterpret_cast<char*>(scratch) + DFLASH_VERIFY_NOALLOC_MAX_ROWS * 8);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(keys, 0, (size_t)bs * B * 8, st) != cudaSuccess) return DFLASH_ERR_CUDA;
+  if (cudaMemsetAsync(tickets, 0, (size_t)bs * 4, st) != cudaSuccess) return DFLASH_ERR_CUDA;
+  const dim3 grid((unsigned)((V + dfl::kVerifyChunk - 1) / dfl::kVerifyChunk), (unsigned)B, (unsigned)bs);
   if (logits_dtype == DFLASH_BF16)
     dfl::verify_kernel<__nv_bfloat16><<<grid, dfl::kVerifyThreads, 0, st>>>(
         (const __nv_bfloat16*)d_logits, d_draft, B, V, keys, tickets, d_accepted, d_next_token);

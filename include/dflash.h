@@ -182,6 +182,32 @@ dflash_status dflash_verify(const void* d_logits, dflash_dtype logits_dtype, con
                             int bs, int B, int V, int* d_accepted, int* d_next_token,
                             void* d_workspace, size_t workspace_bytes, void* stream);
 
+/* Verify for callers that cannot allocate device memory. Same computation,
+ * outputs and bit-exact results as dflash_verify; the pages have no
+ * counterpart, this is a deployment convenience. Some callers may not call
+ * cudaMalloc at all: an inference server's custom-operator interface that hands
+ * a kernel only its input and output buffers, or a serving loop whose memory
+ * pool has already claimed the GPU's free memory for the KV cache, where a raw
+ * cudaMalloc can fail and also synchronises the device, stalling every stream.
+ * This variant keeps its scratch in one fixed array compiled into the library:
+ * DFLASH_VERIFY_NOALLOC_MAX_ROWS 64-bit keys plus DFLASH_VERIFY_NOALLOC_MAX_BATCH
+ * 32-bit tickets (36 KB), present on every GPU that loads the library and held
+ * until the process exits.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current; make that first call before any stream capture.
+ *   - Each call clears the part of the array it uses (cudaMemsetAsync on
+ *     `stream`) before its kernel runs.
+ *   - All calls share the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other host threads) race and
+ *     give wrong results; serialise them.
+ *   - bs > DFLASH_VERIFY_NOALLOC_MAX_BATCH or bs*B > DFLASH_VERIFY_NOALLOC_MAX_ROWS
+ *     is rejected with DFLASH_ERR_ARG and a message on stderr; other arguments
+ *     as for dflash_verify. It allocates nothing. */
+#define DFLASH_VERIFY_NOALLOC_MAX_ROWS 4096
+#define DFLASH_VERIFY_NOALLOC_MAX_BATCH 1024
+dflash_status dflash_verify_noalloc(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft,
+                                    int bs, int B, int V, int* d_accepted, int* d_next_token, void* stream);
+
 /* Per-kernel timing, an instrumentation hook with no counterpart on the pages.
  * While enabled, every kernel this context launches is bracketed by a pair of
  * CUDA events on its stream, tagged with the launch's algorithmic bytes (each

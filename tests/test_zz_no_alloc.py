@@ -1,0 +1,62 @@
+"""dflash_verify_noalloc: the verify entry point for callers that cannot
+allocate device memory (a custom-operator interface that only hands over input
+and output buffers, or a serving loop whose memory pool already owns the GPU's
+free memory, where cudaMalloc can fail and synchronises the device). Its
+scratch is a fixed array inside the library, so this test checks, through the
+C ABI, that two calls in a row give exactly what the allocating dflash_verify
+gives on the same inputs, and that sizes beyond the fixed scratch are refused.
+Kept in a file pytest collects last."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_speculative_cycle_b200 import _binding, dflash_verify_workspace_size, load_library, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(lib, logits, draft, acc, nxt):
+    dt = _binding.DFLASH_BF16 if logits.dtype == torch.bfloat16 else _binding.DFLASH_F32
+    bs, B, V = logits.shape
+    return lib.dflash_verify_noalloc(logits.data_ptr(), dt, draft.data_ptr(), bs, B, V, acc.data_ptr(),
+                                     nxt.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+
+def _allocating(lib, logits, draft, acc, nxt):
+    dt = _binding.DFLASH_BF16 if logits.dtype == torch.bfloat16 else _binding.DFLASH_F32
+    bs, B, V = logits.shape
+    ws = torch.zeros(dflash_verify_workspace_size(bs, B), dtype=torch.uint8, device="cuda")
+    return lib.dflash_verify(logits.data_ptr(), dt, draft.data_ptr(), bs, B, V, acc.data_ptr(), nxt.data_ptr(),
+                             ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+
+
+@pytest.mark.parametrize("dtype,bs,B,V", [(torch.bfloat16, 8, 16, 151936), (torch.float32, 3, 10, 1000)])
+def test_noalloc_verify_matches_dflash_verify_twice_in_a_row(dtype, bs, B, V):
+    lib = load_library()
+    for call in range(2):
+        g = torch.Generator().manual_seed(1000 * call + bs)
+        d = torch.randint(0, V, (bs, B - 1), generator=g, dtype=torch.int32)
+        z, _ = synth.planted_logits(d, V, 2.0, 4.0, seed=call + V, dtype=dtype)
+        z, d = z.cuda(), d.cuda()
+        ref_a = torch.full((bs,), -1, dtype=torch.int32, device="cuda")
+        ref_n = torch.full((bs,), -1, dtype=torch.int32, device="cuda")
+        got_a = torch.full((bs,), -2, dtype=torch.int32, device="cuda")
+        got_n = torch.full((bs,), -2, dtype=torch.int32, device="cuda")
+        assert _allocating(lib, z, d, ref_a, ref_n) == 0
+        assert _noalloc(lib, z, d, got_a, got_n) == 0
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(got_a.cpu().numpy(), ref_a.cpu().numpy())
+        np.testing.assert_array_equal(got_n.cpu().numpy(), ref_n.cpu().numpy())
+
+
+def test_noalloc_verify_refuses_sizes_beyond_its_scratch():
+    lib = load_library()
+    t = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    # bs * B above the fixed capacity: refused on the host, nothing launched
+    assert lib.dflash_verify_noalloc(t.data_ptr(), 1, t.data_ptr(), 257, 16, 10, t.data_ptr(), t.data_ptr(),
+                                     stream) == 1
+    assert lib.dflash_verify_noalloc(t.data_ptr(), 1, t.data_ptr(), 1025, 1, 10, t.data_ptr(), t.data_ptr(),
+                                     stream) == 1
