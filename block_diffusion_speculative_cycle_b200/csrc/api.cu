@@ -21,18 +21,26 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-constexpr int kCountersPerSite = 4096;
-constexpr int kNumSites = 128;
-constexpr size_t kPartialFloats = (size_t)24 << 20;   // split-K partials: 96 MB
 constexpr int kAttnTargetCtas = 296;                   // 2 CTAs per SM on 148 SMs
-
-enum Site { SITE_FC = 0, SITE_KV = 1, SITE_LM = 4, SITE_LAYER0 = 8 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-enum ProfKind { PK_GEMM_TC = 0, PK_GEMM_SIMT, PK_ATTN, PK_EMBED_NORM, PK_RMSNORM, PK_ARGMAX, PK_COPY, PK_COUNT };
-const char* const kProfNames[PK_COUNT] = {"gemm_tc", "gemm_simt", "attention", "embed_norm",
-                                          "rmsnorm", "argmax_finalize", "hidden_copy"};
+// GEMM call sites (profiling tags)
+enum GemmTag { TAG_FC = 0, TAG_KV, TAG_QKV, TAG_O, TAG_GATEUP, TAG_DOWN, TAG_LM, TAG_COUNT };
+enum ProfKind {
+  PK_GEMM_TC = 0,                    // + tag
+  PK_GEMM_SIMT = PK_GEMM_TC + TAG_COUNT,   // + tag
+  PK_ATTN = PK_GEMM_SIMT + TAG_COUNT,
+  PK_EMBED_NORM,
+  PK_RMSNORM,
+  PK_ARGMAX,
+  PK_COPY,
+  PK_COUNT
+};
+const char* const kProfNames[PK_COUNT] = {
+    "gemm_tc:fc", "gemm_tc:kv", "gemm_tc:qkv", "gemm_tc:o", "gemm_tc:gateup", "gemm_tc:down", "gemm_tc:lm",
+    "gemm_simt:fc", "gemm_simt:kv", "gemm_simt:qkv", "gemm_simt:o", "gemm_simt:gateup", "gemm_simt:down",
+    "gemm_simt:lm", "attention", "embed_norm", "rmsnorm", "argmax_finalize", "hidden_copy"};
 
 struct ProfRec {
   int kind;
@@ -65,8 +73,6 @@ struct dflash_ctx {
   void* ao = nullptr;
   void* act = nullptr;
   void* c = nullptr;
-  float* partials = nullptr;
-  int* counters = nullptr;
   unsigned long long* keys = nullptr;
   float* att_o = nullptr;
   float* att_m = nullptr;
@@ -144,9 +150,28 @@ struct GemmSpec {
   const void* w[kMaxSeg] = {};
   int seg_rows[kMaxSeg] = {};
   bool paired = false;
-  int site = 0;
+  int tag = 0;
   EpiParams epi{};
 };
+
+// K splits per output tile (= cluster size). Below one wave of CTAs, split K so
+// the grid fills the SMs; pick the split whose CTA count best fills whole waves.
+int choose_splits(int units, int num_kb, int slots) {
+  if (units >= slots) return 1;
+  int best = 1;
+  double best_eff = (double)units / slots;
+  for (int s = 2; s <= kMaxClusterSplits; ++s) {
+    if (num_kb / s < 2) break;
+    const int ctas = units * s;
+    const int waves = (ctas + slots - 1) / slots;
+    const double eff = (double)ctas / ((double)waves * slots);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
 
 int pow2_at_least(int v) {
   int p = 1;
@@ -182,7 +207,7 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
     case EPI_ARGMAX: out_bytes = (double)g.M * 8; break;
     default: out_bytes = (double)g.M * n_out * es_; break;
   }
-  ProfScope prof(ctx, (!ctx->bf16 || ctx->force_simt) ? PK_GEMM_SIMT : PK_GEMM_TC, st,
+  ProfScope prof(ctx, ((!ctx->bf16 || ctx->force_simt) ? PK_GEMM_SIMT : PK_GEMM_TC) + g.tag, st,
                  w_rows * g.K * es_ + (double)g.M * g.K * es_ + out_bytes, 2.0 * g.M * w_rows * g.K);
 
   if (!ctx->bf16 || ctx->force_simt) {
@@ -210,23 +235,17 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   p.tmem_cols = std::max(32, pow2_at_least(p.m_tile));
   p.num_kb = g.K / 64;
   p.n_tiles = n_tiles;
-  p.n_total = n_tiles * kTileN;
   const int units = n_tiles * p.m_blocks;
   const int per_sm = p.m_tile <= 64 ? 2 : 1;
-  const int target = ctx->num_sms * per_sm;
-  int splits = std::max(1, (target + units - 1) / units);
-  splits = std::min(splits, std::max(1, p.num_kb / 4));
-  while (splits > 1 && (size_t)splits * g.M * p.n_total > kPartialFloats) --splits;
-  const int kbps = (p.num_kb + splits - 1) / splits;
-  p.kb_per_split = kbps;
-  p.splits = (p.num_kb + kbps - 1) / kbps;
+  p.splits = choose_splits(units, p.num_kb, ctx->num_sms * per_sm);
+  p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
   const size_t budget = per_sm == 2 ? 110 * 1024 : 220 * 1024;
   const int sb = kTileN * 64 * 2 + p.m_tile * 128;
   p.stages = (int)std::min<size_t>(8, (budget - 1024) / sb);
   if (p.stages < 2) return DFLASH_ERR_UNSUPPORTED;
-  p.partials = ctx->partials;
-  p.counters = ctx->counters + (size_t)g.site * kCountersPerSite;
-  if (units > kCountersPerSite) return DFLASH_ERR_UNSUPPORTED;
+  // the cluster reduction stages m_tile x 128 fp32 plus one epilogue chunk in the ring's memory
+  if (p.splits > 1 && (size_t)p.stages * sb < (size_t)p.m_tile * kTileN * 4 + kChunkRows * kChunkLd * 4)
+    return DFLASH_ERR_UNSUPPORTED;
   p.use_pdl = ctx->use_pdl ? 1 : 0;
   const int box_w = g.paired ? kTileN / 2 : kTileN;
   const int nmaps = g.paired ? 2 : g.n_seg;
@@ -342,8 +361,6 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   const size_t o_ao = take(R * q_dim(c) * es);
   const size_t o_act = take(R * c.intermediate * es);
   const size_t o_c = take(Rin * c.hidden * es);
-  const size_t o_part = take(ctx->bf16 ? kPartialFloats * 4 : 256);
-  const size_t o_ctr = take((size_t)kNumSites * kCountersPerSite * 4);
   const size_t o_keys = take(R * 8);
   const size_t o_atto = take(ctx->att_rows * c.head_dim * 4);
   const size_t o_attm = take(ctx->att_rows * 4);
@@ -369,8 +386,6 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   ctx->ao = b + o_ao;
   ctx->act = b + o_act;
   ctx->c = b + o_c;
-  ctx->partials = (float*)(b + o_part);
-  ctx->counters = (int*)(b + o_ctr);
   ctx->keys = (unsigned long long*)(b + o_keys);
   ctx->att_o = (float*)(b + o_atto);
   ctx->att_m = (float*)(b + o_attm);
@@ -459,7 +474,7 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
   fcg.n_seg = 1;
   fcg.w[0] = ctx->fc;
   fcg.seg_rows[0] = c.hidden;
-  fcg.site = SITE_FC;
+  fcg.tag = TAG_FC;
   fcg.epi.kind = EPI_STORE;
   fcg.epi.out[0] = ctx->c;
   fcg.epi.ld_out[0] = c.hidden;
@@ -476,7 +491,7 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
     kv.M = M;
     kv.K = c.hidden;
     kv.n_seg = 2 * nl;
-    kv.site = SITE_KV + part;
+    kv.tag = TAG_KV;
     EpiParams& e = kv.epi;
     e.kind = EPI_KV_INJECT;
     for (int i = 0; i < nl; ++i) {
@@ -534,15 +549,17 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   // attention split plan
   const int g = c.n_q_heads / c.n_kv_heads;
   const int T_max = max_ctx + B;
-  int n_splits = std::max(1, (kAttnTargetCtas + bs * c.n_kv_heads - 1) / (bs * c.n_kv_heads));
-  n_splits = std::min(n_splits, (T_max + 31) / 32);
+  // key splits: multiples of the attention kernel's key tile, about one CTA per SM
+  const int key_tile = ctx->bf16 ? 64 : 32;
+  const int target_ctas = ctx->bf16 ? ctx->num_sms : kAttnTargetCtas;
+  int n_splits = std::max(1, (target_ctas + bs * c.n_kv_heads - 1) / (bs * c.n_kv_heads));
+  n_splits = std::min(n_splits, (T_max + key_tile - 1) / key_tile);
   int kps = (T_max + n_splits - 1) / n_splits;
-  kps = (kps + 31) / 32 * 32;
+  kps = (kps + key_tile - 1) / key_tile * key_tile;
   n_splits = (T_max + kps - 1) / kps;
   if ((size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows) return DFLASH_ERR_UNSUPPORTED;
 
   for (int l = 0; l < c.n_layers; ++l) {
-    const int site = SITE_LAYER0 + 4 * l;
     GemmSpec qkv;
     qkv.x = ctx->h;
     qkv.ldx = H;
@@ -555,7 +572,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     qkv.seg_rows[0] = QD;
     qkv.seg_rows[1] = KVD;
     qkv.seg_rows[2] = KVD;
-    qkv.site = site;
+    qkv.tag = TAG_QKV;
     qkv.epi.kind = EPI_QKV;
     qkv.epi.out[0] = ctx->q;
     qkv.epi.out[1] = ctx->kb;
@@ -611,7 +628,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     o.n_seg = 1;
     o.w[0] = ctx->wo[l];
     o.seg_rows[0] = H;
-    o.site = site + 1;
+    o.tag = TAG_O;
     o.epi.kind = EPI_RESID;
     o.epi.x = ctx->x;
     o.epi.ldx = H;
@@ -632,7 +649,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     gu.w[0] = ctx->wg[l];
     gu.w[1] = ctx->wu[l];
     gu.seg_rows[0] = gu.seg_rows[1] = c.intermediate;
-    gu.site = site + 2;
+    gu.tag = TAG_GATEUP;
     gu.epi.kind = EPI_SWIGLU;
     gu.epi.out[0] = ctx->act;
     gu.epi.ld_out[0] = c.intermediate;
@@ -646,7 +663,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     dn.n_seg = 1;
     dn.w[0] = ctx->wd[l];
     dn.seg_rows[0] = H;
-    dn.site = site + 3;
+    dn.tag = TAG_DOWN;
     dn.epi.kind = EPI_RESID;
     dn.epi.x = ctx->x;
     dn.epi.ldx = H;
@@ -677,7 +694,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   lm.n_seg = 1;
   lm.w[0] = ctx->lm_head;
   lm.seg_rows[0] = c.vocab;
-  lm.site = SITE_LM;
+  lm.tag = TAG_LM;
   lm.epi.kind = EPI_ARGMAX;
   lm.epi.keys = ctx->keys;
   DFL_CHECK(run_gemm(ctx, lm, st));

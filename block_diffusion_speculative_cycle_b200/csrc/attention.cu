@@ -120,7 +120,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
   }
 }
 
-// One warp per (block row, query head): merge the splits that hold keys.
+// One warp per (block row, query head): merge the splits that hold keys. Lanes
+// own splits for the max and the weights; the weighted sum of the split outputs
+// then reads each split's row with all lanes (d/32 values per lane).
 template <typename OT, int D>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p, OT* out) {
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
@@ -135,21 +137,32 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p, OT*
   const int used = min(p.n_splits, (P + p.B + p.kps - 1) / p.kps);
   const size_t base = (size_t)(b * p.n_kv + h) * p.n_splits * nr + r;
   float M = -INFINITY;
-  for (int s = 0; s < used; ++s) M = fmaxf(M, p.part_m[base + (size_t)s * nr]);
-  float L = 0.f, acc[D / 32];
+  for (int s = lane; s < used; s += 32) M = fmaxf(M, p.part_m[base + (size_t)s * nr]);
+  M = warp_max(M);
+  float L = 0.f;
+  for (int s = lane; s < used; s += 32) {
+    const size_t idx = base + (size_t)s * nr;
+    L += p.part_l[idx] * expf(p.part_m[idx] - M);
+  }
+  L = warp_sum(L);
+  const float invL = 1.f / L;
+  float acc[D / 32];
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
-  for (int s = 0; s < used; ++s) {
-    const size_t idx = base + (size_t)s * nr;
-    const float w = expf(p.part_m[idx] - M);
-    L += p.part_l[idx] * w;
+  for (int s0 = 0; s0 < used; s0 += 32) {
+    const int sl = s0 + lane;
+    const float wl = sl < used ? expf(p.part_m[base + (size_t)sl * nr] - M) * invL : 0.f;
+    const int n = min(32, used - s0);
+#pragma unroll 4
+    for (int k = 0; k < n; ++k) {
+      const float w = __shfl_sync(0xffffffffu, wl, k);
+      const float* o = p.part_o + (base + (size_t)(s0 + k) * nr) * D;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(w, p.part_o[idx * D + lane + 32 * c], acc[c]);
+      for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(w, o[lane + 32 * c], acc[c]);
+    }
   }
-  const float inv = 1.f / L;
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c)
-    out[(size_t)m_row * p.n_q * D + j * D + lane + 32 * c] = from_f32<OT>(acc[c] * inv);
+  for (int c = 0; c < D / 32; ++c) out[(size_t)m_row * p.n_q * D + j * D + lane + 32 * c] = from_f32<OT>(acc[c]);
 }
 
 template <typename T, int D, int RPW>
@@ -179,10 +192,12 @@ static cudaError_t launch_split_rpw(const AttnParams& p, cudaStream_t st) {
 
 cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st) {
   cudaError_t e;
-  if (p.d == 128)
-    e = in_bf16 ? launch_split_rpw<__nv_bfloat16, 128>(p, st) : launch_split_rpw<float, 128>(p, st);
+  if (in_bf16)
+    e = launch_attn_mma(p, st);
+  else if (p.d == 128)
+    e = launch_split_rpw<float, 128>(p, st);
   else
-    e = in_bf16 ? launch_split_rpw<__nv_bfloat16, 64>(p, st) : launch_split_rpw<float, 64>(p, st);
+    e = launch_split_rpw<float, 64>(p, st);
   if (e != cudaSuccess) return e;
   const int warps = p.bs * p.B * p.n_q;
   const dim3 grid((warps + 7) / 8);

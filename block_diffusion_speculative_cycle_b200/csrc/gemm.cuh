@@ -171,18 +171,16 @@ struct alignas(64) GemmTcParams {
   int m_blocks;
   int tmem_cols;
   int num_kb;                  // K / 64
-  int splits;
+  int splits;                  // K splits = cluster size (1..8)
   int kb_per_split;
   int n_tiles;
-  int n_total;                 // output tile rows in total (n_tiles * 128)
   int stages;
-  float* partials;             // [splits, M, n_total] when splits > 1
-  int* counters;               // [m_blocks * n_tiles], zero between launches
   int use_pdl;
 };
 
 void launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t st);
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st);
 size_t gemm_tc_smem_bytes(int m_tile, int stages);
+constexpr int kMaxClusterSplits = 8;
 
 }  // namespace dfl

@@ -8,13 +8,19 @@
 //   warp 0       TMA producer (one elected lane), ring of `stages` stages
 //   warp 1       TMEM owner + MMA issuer (one elected lane)
 //   warps 2..5   epilogue: TMEM -> registers -> smem chunk -> fused epilogue
-// Split-K: every split writes fp32 partials; the last CTA to finish a tile
-// (atomic ticket) sums the splits in split order and runs the epilogue, so the
-// result does not depend on CTA timing.
+// Split-K across a thread-block cluster: the `splits` CTAs of one output tile
+// form a cluster, each reduces its own K range into TMEM, stages the fp32
+// accumulator in its shared memory, and after a cluster barrier CTA r sums rows
+// [r*m/splits, (r+1)*m/splits) over all CTAs' staging through distributed shared
+// memory, in rank order (deterministic), then runs the fused epilogue on them.
 // Every mbarrier wait is bounded; on a timeout the CTA flags ST_TIMEOUT, lets
 // its copies in flight land, frees TMEM and returns.
+#include <cooperative_groups.h>
+
 #include "gemm.cuh"
 #include "sm100.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace dfl {
 
@@ -37,11 +43,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   __shared__ int s_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // blockIdx.x = ((tile * m_blocks) + mb) * splits + split; split = rank in the cluster
   int id = blockIdx.x;
-  const int mb = id % p.m_blocks;
-  id /= p.m_blocks;
   const int split = id % p.splits;
-  const int tile = id / p.splits;
+  id /= p.splits;
+  const int mb = id % p.m_blocks;
+  const int tile = id / p.m_blocks;
   const int kb0 = split * p.kb_per_split;
   const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
   const int nkb = kb1 - kb0;
@@ -155,41 +162,54 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           named_bar_sync(1, 128);
         }
       } else {
-        const size_t col = (size_t)tile * kTileN + t;
+        // stage this split's accumulator: stage[m][t], m < rows_here
+        float* stage = reinterpret_cast<float*>(base);
         for (int c0 = 0; c0 < rows_here; c0 += kChunkRows) {
           tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, v);
-          const int nr = min(kChunkRows, rows_here - c0);
-          for (int j = 0; j < nr; ++j)
-            p.partials[((size_t)split * p.M + row0 + c0 + j) * p.n_total + col] = v[j];
-        }
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (t == 0) {
-          int* ctr = p.counters + (size_t)mb * p.n_tiles + tile;
-          const int prev = atomicAdd(ctr, 1);
-          const int last = prev == p.splits - 1;
-          if (last) atomicExch(ctr, 0);
-          s_flag = last ? 2 : 0;
-        }
-        named_bar_sync(1, 128);
-        if (s_flag == 2) {
-          __threadfence();
-          for (int c0 = 0; c0 < rows_here; c0 += kChunkRows) {
-            const int nr = min(kChunkRows, rows_here - c0);
-            for (int j = 0; j < nr; ++j) {
-              float sum = 0.f;
-              for (int s = 0; s < p.splits; ++s)
-                sum += __ldcg(p.partials + ((size_t)s * p.M + row0 + c0 + j) * p.n_total + col);
-              chunk[j * kChunkLd + t] = sum;
-            }
-            named_bar_sync(1, 128);
-            epilogue_chunk(p.epi, tile, row0 + c0, nr, chunk, t);
-            named_bar_sync(1, 128);
-          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < rows_here) stage[(c0 + j) * kTileN + t] = v[j];
         }
       }
+    } else if (p.splits > 1) {
+      // no K range (or a timed-out wait): contribute zeros
+      float* stage = reinterpret_cast<float*>(base);
+      for (int m = 0; m < rows_here; ++m) stage[m * kTileN + t] = 0.f;
     }
     tc_fence_before();
+  }
+  if (p.splits > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();   // every split's staging is written
+    if (warp >= 2) {
+      const int t = (warp & 3) * 32 + lane;
+      const int row0 = mb * p.m_tile;
+      const int rows_here = min(p.m_tile, p.M - row0);
+      const int per = (rows_here + p.splits - 1) / p.splits;
+      const int r_lo = split * per, r_hi = min(rows_here, r_lo + per);
+      float* stage = reinterpret_cast<float*>(base);
+      float* chunk = stage + (size_t)p.m_tile * kTileN;
+      const float* rem[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) rem[s] = s < p.splits ? cluster.map_shared_rank(stage, s) : stage;
+      for (int c0 = r_lo; c0 < r_hi; c0 += kChunkRows) {
+        const int nr = min(kChunkRows, r_hi - c0);
+        for (int j = 0; j < nr; ++j) {
+          const int off = (c0 + j) * kTileN + t;
+          float part[8];
+#pragma unroll
+          for (int s = 0; s < 8; ++s) part[s] = s < p.splits ? rem[s][off] : 0.f;
+          float sum = 0.f;
+#pragma unroll
+          for (int s = 0; s < 8; ++s) sum += part[s];
+          chunk[j * kChunkLd + t] = sum;
+        }
+        named_bar_sync(1, 128);
+        epilogue_chunk(p.epi, tile, row0 + c0, nr, chunk, t);
+        named_bar_sync(1, 128);
+      }
+    }
+    cluster.sync();   // no CTA leaves while a peer may still read its staging
   }
   __syncthreads();
   if (warp == 1) {
@@ -213,11 +233,15 @@ cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = p.use_pdl ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)p.splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.splits > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, gemm_tc_kernel, p);
 }
 

@@ -25,6 +25,9 @@ struct AttnParams {
   int* status;
 };
 
+// Tensor-core (bf16) split-KV attention partials; key splits must be multiples of 64.
+cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st);
+
 // Split-KV attention partials, then the log-sum-exp merge into out [R, n_q*d].
 cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st);
 

@@ -22,22 +22,52 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return t;
 }
 
-// RMSNorm of one fp32 row held in x_row, written to h_row (and y_row if given).
-template <typename HT>
-__device__ __forceinline__ void norm_row(const float* x_row, int H, const float* gain, float eps, HT* h_row,
-                                         float* y_row, float* red) {
+// Load x[0..H) (fp32) into registers as float4, VPT per thread; returns the sum of squares.
+template <int VPT>
+__device__ __forceinline__ float load_row(const float* x_row, int H, float4* v) {
+  const float4* xr = reinterpret_cast<const float4*>(x_row);
+  const int n4 = H >> 2;
   float ss = 0.f;
-  for (int c = threadIdx.x; c < H; c += blockDim.x) ss = fmaf(x_row[c], x_row[c], ss);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = i * blockDim.x + threadIdx.x;
+    v[i] = idx < n4 ? xr[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+  return ss;
+}
+
+__device__ __forceinline__ void store4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+
+// h = v * rsqrt(ss/H + eps) * gain (and an fp32 copy into y if given)
+template <int VPT, typename HT>
+__device__ __forceinline__ void norm_store(const float4* v, float ss, int H, const float* gain, float eps, HT* h_row,
+                                           float* y_row, float* red) {
   ss = block_sum(ss, red);
   const float rstd = rsqrtf(ss / (float)H + eps);
-  for (int c = threadIdx.x; c < H; c += blockDim.x) {
-    const float y = x_row[c] * rstd * gain[c];
-    h_row[c] = from_f32<HT>(y);
-    if (y_row) y_row[c] = y;
+  const float4* g4 = reinterpret_cast<const float4*>(gain);
+  const int n4 = H >> 2;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = i * blockDim.x + threadIdx.x;
+    if (idx < n4) {
+      const float4 g = g4[idx];
+      const float4 y = make_float4(v[i].x * rstd * g.x, v[i].y * rstd * g.y, v[i].z * rstd * g.z, v[i].w * rstd * g.w);
+      store4(h_row + 4 * idx, y);
+      if (y_row) store4(y_row + 4 * idx, y);
+    }
   }
 }
 
-template <typename ET, typename HT>
+template <int VPT, typename ET, typename HT>
 __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const ET* embed, const int* anchor, int mask_id,
                                                                   int B, int V, int H, const float* gain,
                                                                   float eps, float* x, HT* h, int* status) {
@@ -48,18 +78,34 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const ET* embe
     if (threadIdx.x == 0) flag_error(status, ST_BAD_TOKEN);
     tok = 0;
   }
-  float* xr = x + (size_t)m * H;
-  for (int c = threadIdx.x; c < H; c += blockDim.x) xr[c] = to_f32(embed[(size_t)tok * H + c]);
-  __syncthreads();
-  norm_row(xr, H, gain, eps, h + (size_t)m * H, nullptr, red);
+  const ET* er = embed + (size_t)tok * H;
+  float4 v[VPT];
+  float ss = 0.f;
+  const int n4 = H >> 2;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = i * blockDim.x + threadIdx.x;
+    v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (idx < n4)
+      v[i] = make_float4(to_f32(er[4 * idx]), to_f32(er[4 * idx + 1]), to_f32(er[4 * idx + 2]), to_f32(er[4 * idx + 3]));
+  }
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = i * blockDim.x + threadIdx.x;
+    if (idx < n4) store4(x + (size_t)m * H + 4 * idx, v[i]);
+    ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+  }
+  norm_store<VPT>(v, ss, H, gain, eps, h + (size_t)m * H, nullptr, red);
 }
 
-template <typename HT>
+template <int VPT, typename HT>
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* x, int H, const float* gain, float eps,
                                                                HT* h, float* y) {
   __shared__ float red[32];
   const int m = blockIdx.x;
-  norm_row(x + (size_t)m * H, H, gain, eps, h + (size_t)m * H, y ? y + (size_t)m * H : nullptr, red);
+  float4 v[VPT];
+  const float ss = load_row<VPT>(x + (size_t)m * H, H, v);
+  norm_store<VPT>(v, ss, H, gain, eps, h + (size_t)m * H, y ? y + (size_t)m * H : nullptr, red);
 }
 
 __global__ void argmax_finalize_kernel(unsigned long long* keys, int bs, int B, int* draft) {
@@ -71,29 +117,50 @@ __global__ void argmax_finalize_kernel(unsigned long long* keys, int bs, int B, 
   keys[e] = 0ull;
 }
 
+template <int VPT>
+static void embed_norm_vpt(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
+                           int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
+                           cudaStream_t st) {
+  if (embed_bf16 && h_bf16)
+    embed_norm_kernel<VPT, __nv_bfloat16, __nv_bfloat16><<<R, kNormThreads, 0, st>>>(
+        (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, status);
+  else if (!embed_bf16 && !h_bf16)
+    embed_norm_kernel<VPT, float, float><<<R, kNormThreads, 0, st>>>((const float*)embed, anchor, mask_id, B, V, H,
+                                                                     gain, eps, x, (float*)h, status);
+  else if (embed_bf16)
+    embed_norm_kernel<VPT, __nv_bfloat16, float><<<R, kNormThreads, 0, st>>>(
+        (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (float*)h, status);
+  else
+    embed_norm_kernel<VPT, float, __nv_bfloat16><<<R, kNormThreads, 0, st>>>(
+        (const float*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, status);
+}
+
 void launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
                        int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
                        cudaStream_t st) {
-  if (embed_bf16 && h_bf16)
-    embed_norm_kernel<__nv_bfloat16, __nv_bfloat16><<<R, kNormThreads, 0, st>>>(
-        (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, status);
-  else if (!embed_bf16 && !h_bf16)
-    embed_norm_kernel<float, float><<<R, kNormThreads, 0, st>>>((const float*)embed, anchor, mask_id, B, V, H, gain,
-                                                                eps, x, (float*)h, status);
-  else if (embed_bf16)
-    embed_norm_kernel<__nv_bfloat16, float><<<R, kNormThreads, 0, st>>>(
-        (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (float*)h, status);
+  const int vpt = (H / 4 + kNormThreads - 1) / kNormThreads;
+  if (vpt <= 1) embed_norm_vpt<1>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st);
+  else if (vpt <= 2) embed_norm_vpt<2>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st);
+  else if (vpt <= 4) embed_norm_vpt<4>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st);
+  else embed_norm_vpt<8>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st);
+}
+
+template <int VPT>
+static void rmsnorm_vpt(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
+                        cudaStream_t st) {
+  if (h_bf16)
+    rmsnorm_kernel<VPT, __nv_bfloat16><<<R, kNormThreads, 0, st>>>(x, H, gain, eps, (__nv_bfloat16*)h, y);
   else
-    embed_norm_kernel<float, __nv_bfloat16><<<R, kNormThreads, 0, st>>>(
-        (const float*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, status);
+    rmsnorm_kernel<VPT, float><<<R, kNormThreads, 0, st>>>(x, H, gain, eps, (float*)h, y);
 }
 
 void launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
                     cudaStream_t st) {
-  if (h_bf16)
-    rmsnorm_kernel<__nv_bfloat16><<<R, kNormThreads, 0, st>>>(x, H, gain, eps, (__nv_bfloat16*)h, y);
-  else
-    rmsnorm_kernel<float><<<R, kNormThreads, 0, st>>>(x, H, gain, eps, (float*)h, y);
+  const int vpt = (H / 4 + kNormThreads - 1) / kNormThreads;
+  if (vpt <= 1) rmsnorm_vpt<1>(x, R, H, gain, eps, h, h_bf16, y, st);
+  else if (vpt <= 2) rmsnorm_vpt<2>(x, R, H, gain, eps, h, h_bf16, y, st);
+  else if (vpt <= 4) rmsnorm_vpt<4>(x, R, H, gain, eps, h, h_bf16, y, st);
+  else rmsnorm_vpt<8>(x, R, H, gain, eps, h, h_bf16, y, st);
 }
 
 void launch_argmax_finalize(unsigned long long* keys, int bs, int B, int* draft, cudaStream_t st) {
