@@ -83,6 +83,7 @@ struct dflash_ctx {
   bool prof = false;
   std::vector<ProfRec> recs;
   std::map<std::tuple<const void*, long long, long long, long long, int>, CUtensorMap> maps;
+  std::map<std::pair<int, int>, int> cluster_cap;   // (m_tile*16 + stages, splits) -> co-resident clusters
 };
 
 namespace {
@@ -154,23 +155,24 @@ struct GemmSpec {
   EpiParams epi{};
 };
 
-// K splits per output tile (= cluster size). Below one wave of CTAs, split K so
-// the grid fills the SMs; pick the split whose CTA count best fills whole waves.
-int choose_splits(int units, int num_kb, int slots) {
-  if (units >= slots) return 1;
-  int best = 1;
-  double best_eff = (double)units / slots;
-  for (int s = 2; s <= kMaxClusterSplits; ++s) {
-    if (num_kb / s < 2) break;
-    const int ctas = units * s;
-    const int waves = (ctas + slots - 1) / slots;
-    const double eff = (double)ctas / ((double)waves * slots);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = s;
+// K splits per output tile (= cluster size): the largest split count whose
+// grid still fits on the GPU in one wave (every CTA co-resident), so the weight
+// stream runs on as many SMs as possible without a tail wave.
+int choose_splits(dflash_ctx* ctx, int units, int num_kb, int m_tile, int stages) {
+  for (int s = kMaxClusterSplits; s >= 2; --s) {
+    if (num_kb / s < 2) continue;
+    const auto key = std::make_pair(m_tile * 16 + stages, s);
+    auto it = ctx->cluster_cap.find(key);
+    int cap;
+    if (it != ctx->cluster_cap.end()) {
+      cap = it->second;
+    } else {
+      cap = gemm_tc_max_active_clusters(m_tile, stages, s);
+      ctx->cluster_cap[key] = cap;
     }
+    if (units <= cap) return s;
   }
-  return best;
+  return 1;
 }
 
 int pow2_at_least(int v) {
@@ -221,8 +223,7 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
     p.w_bf16 = ctx->bf16 ? 1 : 0;
     p.x_bf16 = ctx->bf16 ? 1 : 0;
     p.epi = e;
-    launch_gemm_simt(p, n_tiles, st);
-    return cuda_status(cudaGetLastError(), "gemm_simt launch");
+    return cuda_status(launch_gemm_simt(p, n_tiles, st, ctx->use_pdl), "gemm_simt launch");
   }
 
   GemmTcParams p;
@@ -237,12 +238,12 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   p.n_tiles = n_tiles;
   const int units = n_tiles * p.m_blocks;
   const int per_sm = p.m_tile <= 64 ? 2 : 1;
-  p.splits = choose_splits(units, p.num_kb, ctx->num_sms * per_sm);
-  p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
   const size_t budget = per_sm == 2 ? 110 * 1024 : 220 * 1024;
   const int sb = kTileN * 64 * 2 + p.m_tile * 128;
   p.stages = (int)std::min<size_t>(8, (budget - 1024) / sb);
   if (p.stages < 2) return DFLASH_ERR_UNSUPPORTED;
+  p.splits = choose_splits(ctx, units, p.num_kb, p.m_tile, p.stages);
+  p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
   // the cluster reduction stages m_tile x 128 fp32 plus one epilogue chunk in the ring's memory
   if (p.splits > 1 && (size_t)p.stages * sb < (size_t)p.m_tile * kTileN * 4 + kChunkRows * kChunkLd * 4)
     return DFLASH_ERR_UNSUPPORTED;
@@ -306,7 +307,7 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   const char* env = std::getenv("DFLASH_FORCE_SIMT");
   ctx->force_simt = env && env[0] == '1';
   env = std::getenv("DFLASH_PDL");
-  ctx->use_pdl = env && env[0] == '1';
+  ctx->use_pdl = !(env && env[0] == '0');
   int dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev);
@@ -539,20 +540,21 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   const double es = (double)esize(ctx);
   {
     ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
-    launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, B, R, c.vocab, H,
-                      c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps, ctx->x, ctx->h, hb,
-                      ctx->status, st);
+    DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, B, R, c.vocab, H,
+                                            c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps,
+                                            ctx->x, ctx->h, hb, ctx->status, st, ctx->use_pdl),
+                          "embed_norm launch"));
   }
-  if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
   const double norm_bytes = (double)R * H * (4 + es);
 
   // attention split plan
   const int g = c.n_q_heads / c.n_kv_heads;
   const int T_max = max_ctx + B;
-  // key splits: multiples of the attention kernel's key tile, about one CTA per SM
+  // key splits: multiples of the attention kernel's key tile, about two CTAs per SM;
+  // the bf16 kernel's splits of one (request, KV head) form one cluster
   const int key_tile = ctx->bf16 ? 64 : 32;
-  const int target_ctas = ctx->bf16 ? ctx->num_sms : kAttnTargetCtas;
-  int n_splits = std::max(1, (target_ctas + bs * c.n_kv_heads - 1) / (bs * c.n_kv_heads));
+  int n_splits = std::max(1, (kAttnTargetCtas + bs * c.n_kv_heads - 1) / (bs * c.n_kv_heads));
+  if (ctx->bf16) n_splits = std::min(n_splits, kMaxAttnCluster);
   n_splits = std::min(n_splits, (T_max + key_tile - 1) / key_tile);
   int kps = (T_max + n_splits - 1) / n_splits;
   kps = (kps + key_tile - 1) / key_tile * key_tile;
@@ -617,7 +619,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
       const double kvb = (double)bs * max_ctx * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;
       const double fl = 4.0 * bs * B * (double)(max_ctx + B) * QD;
       ProfScope prof(ctx, PK_ATTN, st, kvb, fl);
-      DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, hb, hb, st), "attention launch"));
+      DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, hb, hb, st, ctx->use_pdl), "attention launch"));
     }
 
     GemmSpec o;
@@ -636,7 +638,9 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
 
     {
       ProfScope prof(ctx, PK_RMSNORM, st, norm_bytes, 0);
-      launch_rmsnorm(ctx->x, R, H, ctx->mlp_norm[l], c.rms_eps, ctx->h, hb, nullptr, st);
+      DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->mlp_norm[l], c.rms_eps, ctx->h, hb, nullptr, st,
+                                           ctx->use_pdl),
+                            "rmsnorm launch"));
     }
 
     GemmSpec gu;
@@ -678,13 +682,17 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     const bool last = l + 1 == c.n_layers;
     {
       ProfScope prof(ctx, PK_RMSNORM, st, norm_bytes, 0);
-      launch_rmsnorm(ctx->x, R, H, last ? ctx->final_norm : ctx->attn_norm[l + 1], c.rms_eps, ctx->h, hb,
-                     last && d_hidden_out ? d_hidden_out + (size_t)c.n_layers * layer_stride : nullptr, st);
+      DFL_CHECK(cuda_status(
+          launch_rmsnorm(ctx->x, R, H, last ? ctx->final_norm : ctx->attn_norm[l + 1], c.rms_eps, ctx->h, hb,
+                         last && d_hidden_out ? d_hidden_out + (size_t)c.n_layers * layer_stride : nullptr, st,
+                         ctx->use_pdl),
+          "rmsnorm launch"));
     }
   }
   if (c.n_layers == 0 && d_hidden_out)
-    launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, ctx->h, hb, d_hidden_out, st);
-  if (cudaGetLastError() != cudaSuccess) return DFLASH_ERR_CUDA;
+    DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, ctx->h, hb, d_hidden_out, st,
+                                         ctx->use_pdl),
+                          "rmsnorm launch"));
 
   GemmSpec lm;
   lm.x = ctx->h;
@@ -700,7 +708,8 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   DFL_CHECK(run_gemm(ctx, lm, st));
   {
     ProfScope prof(ctx, PK_ARGMAX, st, (double)R * 8 * 2 + (double)bs * (B - 1) * 4, 0);
-    launch_argmax_finalize(ctx->keys, bs, B, d_draft, st);
+    DFL_CHECK(cuda_status(launch_argmax_finalize(ctx->keys, bs, B, d_draft, st, ctx->use_pdl),
+                          "argmax_finalize launch"));
   }
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+  return DFLASH_OK;
 }

@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
   const T* vb = reinterpret_cast<const T*>(p.vblk);
   const T* kc = reinterpret_cast<const T*>(p.kc);
   const T* vc = reinterpret_cast<const T*>(p.vc);
+  grid_dep_wait();
+  grid_dep_launch();
 
   int P = p.ctx_len[b];
   if (P < 0 || P > p.max_ctx) {
@@ -125,6 +127,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
 // then reads each split's row with all lanes (d/32 values per lane).
 template <typename OT, int D>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p, OT* out) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int R = p.bs * p.B;
   if (gw >= R * p.n_q) return;
@@ -166,7 +170,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p, OT*
 }
 
 template <typename T, int D, int RPW>
-static cudaError_t launch_split(const AttnParams& p, cudaStream_t st) {
+static cudaError_t launch_split(const AttnParams& p, cudaStream_t st, bool pdl) {
   const int nr = p.g * p.B;
   const size_t smem = ((size_t)nr * D + 2 * kKeyTile * (D + 1)) * sizeof(float);
   static size_t attr_bytes = 0;
@@ -176,39 +180,28 @@ static cudaError_t launch_split(const AttnParams& p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_bytes = smem;
   }
-  attn_split_kernel<T, D, RPW><<<dim3(p.n_splits, p.n_kv, p.bs), kAttnThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(attn_split_kernel<T, D, RPW>, dim3(p.n_splits, p.n_kv, p.bs), dim3(kAttnThreads), smem, st,
+                       pdl, p);
 }
 
 template <typename T, int D>
-static cudaError_t launch_split_rpw(const AttnParams& p, cudaStream_t st) {
+static cudaError_t launch_split_rpw(const AttnParams& p, cudaStream_t st, bool pdl) {
   const int rpw = (p.g * p.B + 7) / 8;
-  if (rpw <= 1) return launch_split<T, D, 1>(p, st);
-  if (rpw <= 2) return launch_split<T, D, 2>(p, st);
-  if (rpw <= 4) return launch_split<T, D, 4>(p, st);
-  if (rpw <= 8) return launch_split<T, D, 8>(p, st);
-  return launch_split<T, D, 16>(p, st);
+  if (rpw <= 1) return launch_split<T, D, 1>(p, st, pdl);
+  if (rpw <= 2) return launch_split<T, D, 2>(p, st, pdl);
+  if (rpw <= 4) return launch_split<T, D, 4>(p, st, pdl);
+  if (rpw <= 8) return launch_split<T, D, 8>(p, st, pdl);
+  return launch_split<T, D, 16>(p, st, pdl);
 }
 
-cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st) {
-  cudaError_t e;
-  if (in_bf16)
-    e = launch_attn_mma(p, st);
-  else if (p.d == 128)
-    e = launch_split_rpw<float, 128>(p, st);
-  else
-    e = launch_split_rpw<float, 64>(p, st);
+cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st, bool pdl) {
+  if (in_bf16 && out_bf16) return launch_attn_cluster(p, out, st, pdl);
+  cudaError_t e = p.d == 128 ? launch_split_rpw<float, 128>(p, st, pdl) : launch_split_rpw<float, 64>(p, st, pdl);
   if (e != cudaSuccess) return e;
   const int warps = p.bs * p.B * p.n_q;
-  const dim3 grid((warps + 7) / 8);
-  if (p.d == 128) {
-    if (out_bf16) attn_merge_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(p, (__nv_bfloat16*)out);
-    else attn_merge_kernel<float, 128><<<grid, 256, 0, st>>>(p, (float*)out);
-  } else {
-    if (out_bf16) attn_merge_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(p, (__nv_bfloat16*)out);
-    else attn_merge_kernel<float, 64><<<grid, 256, 0, st>>>(p, (float*)out);
-  }
-  return cudaGetLastError();
+  const dim3 grid((warps + 7) / 8), block(256);
+  if (p.d == 128) return launch_kernel(attn_merge_kernel<float, 128>, grid, block, 0, st, pdl, p, (float*)out);
+  return launch_kernel(attn_merge_kernel<float, 64>, grid, block, 0, st, pdl, p, (float*)out);
 }
 
 }  // namespace dfl

@@ -178,7 +178,9 @@ struct alignas(64) GemmTcParams {
   int use_pdl;
 };
 
-void launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t st);
+cudaError_t launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t st, bool pdl);
+// Clusters of `splits` CTAs of this GEMM configuration that fit on the GPU at once.
+int gemm_tc_max_active_clusters(int m_tile, int stages, int splits);
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st);
 size_t gemm_tc_smem_bytes(int m_tile, int stages);
 constexpr int kMaxClusterSplits = 8;

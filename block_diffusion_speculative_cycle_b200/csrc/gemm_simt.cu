@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(128) gemm_simt_kernel(const GemmSimtParams p) 
   const int nrows = min(kChunkRows, p.M - row0);
   const WT* const* wseg = reinterpret_cast<const WT* const*>(p.w);
   const XT* x = reinterpret_cast<const XT*>(p.x);
+  grid_dep_wait();
+  grid_dep_launch();
 
   // weight row pointer for tile row r
   auto wrow = [&](int r) -> const WT* {
@@ -57,16 +59,12 @@ __global__ void __launch_bounds__(128) gemm_simt_kernel(const GemmSimtParams p) 
   epilogue_chunk(p.epi, tile, row0, nrows, chunk, t);
 }
 
-void launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t st) {
-  dim3 grid((unsigned)n_tiles, (unsigned)((p.M + kChunkRows - 1) / kChunkRows));
-  if (p.w_bf16 && p.x_bf16)
-    gemm_simt_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 128, 0, st>>>(p);
-  else if (!p.w_bf16 && !p.x_bf16)
-    gemm_simt_kernel<float, float><<<grid, 128, 0, st>>>(p);
-  else if (p.w_bf16)
-    gemm_simt_kernel<__nv_bfloat16, float><<<grid, 128, 0, st>>>(p);
-  else
-    gemm_simt_kernel<float, __nv_bfloat16><<<grid, 128, 0, st>>>(p);
+cudaError_t launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t st, bool pdl) {
+  const dim3 grid((unsigned)n_tiles, (unsigned)((p.M + kChunkRows - 1) / kChunkRows)), block(128);
+  if (p.w_bf16 && p.x_bf16) return launch_kernel(gemm_simt_kernel<__nv_bfloat16, __nv_bfloat16>, grid, block, 0, st, pdl, p);
+  if (!p.w_bf16 && !p.x_bf16) return launch_kernel(gemm_simt_kernel<float, float>, grid, block, 0, st, pdl, p);
+  if (p.w_bf16) return launch_kernel(gemm_simt_kernel<__nv_bfloat16, float>, grid, block, 0, st, pdl, p);
+  return launch_kernel(gemm_simt_kernel<float, __nv_bfloat16>, grid, block, 0, st, pdl, p);
 }
 
 }  // namespace dfl

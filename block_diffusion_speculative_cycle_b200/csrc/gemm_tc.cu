@@ -91,13 +91,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const int seg = p.paired ? 0 : seg_of_tile(p.epi, tile);
       const int wrow = p.paired ? tile * (kTileN / 2) : (tile - p.epi.seg_tile_begin[seg]) * kTileN;
       const uint32_t tx = (uint32_t)sbytes;
-      int issued = 0;
-      bool ok = true;
-      // Activations come from the previous kernel; weights do not.
+      const int pre = min(nkb, S);
+      // The first `pre` stages' weight tiles do not depend on the previous kernel:
+      // issue them before waiting for it (programmatic dependent launch).
+      for (int i = 0; i < pre; ++i) {
+        uint8_t* a = base + (size_t)i * sbytes;
+        const int kc = (kb0 + i) * 64;
+        mbar_arrive_expect_tx(&full_bar[i], tx);
+        if (p.paired) {
+          tma_load_2d(a, &p.wmap[0], &full_bar[i], kc, wrow, pol_w);
+          tma_load_2d(a + kABytes / 2, &p.wmap[1], &full_bar[i], kc, wrow, pol_w);
+        } else {
+          tma_load_2d(a, &p.wmap[seg], &full_bar[i], kc, wrow, pol_w);
+        }
+      }
       grid_dep_wait();
-      for (int i = 0; i < nkb && ok; ++i) {
+      for (int i = 0; i < pre; ++i)
+        tma_load_2d(base + (size_t)i * sbytes + kABytes, &p.xmap, &full_bar[i], (kb0 + i) * 64, mb * p.m_tile, pol_x);
+      int issued = pre;
+      bool ok = true;
+      for (int i = pre; i < nkb && ok; ++i) {
         const int s = i % S;
-        if (i >= S) ok = mbar_wait(&empty_bar[s], ((i / S) & 1) ^ 1, status);
+        ok = mbar_wait(&empty_bar[s], ((i / S) & 1) ^ 1, status);
         if (!ok) break;
         uint8_t* a = base + (size_t)s * sbytes;
         uint8_t* b = a + kABytes;
@@ -112,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         tma_load_2d(b, &p.xmap, &full_bar[s], kc, mb * p.m_tile, pol_x);
         ++issued;
       }
+      grid_dep_launch();
       // Let every copy this CTA issued land before the CTA can exit.
       for (int i = max(0, issued - S); i < issued; ++i) mbar_wait(&full_bar[i % S], (i / S) & 1, status);
     }
@@ -143,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int row0 = mb * p.m_tile;
     const int rows_here = min(p.m_tile, p.M - row0);
     float* chunk = reinterpret_cast<float*>(base);
+    grid_dep_wait();   // epilogue reads / writes data shared with the previous kernel
     bool ok = nkb > 0 ? mbar_wait(&acc_bar, 0, status) : true;
     if (!ok) s_flag = 1;
     named_bar_sync(1, 128);
@@ -216,6 +233,33 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     tc_fence_after();
     tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
   }
+}
+
+int gemm_tc_max_active_clusters(int m_tile, int stages, int splits) {
+  const size_t smem = gemm_tc_smem_bytes(m_tile, stages);
+  static size_t attr_bytes_q = 0;
+  if (smem > attr_bytes_q) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return 0;
+    attr_bytes_q = smem;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)splits * 64);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st) {

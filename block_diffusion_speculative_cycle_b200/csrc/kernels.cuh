@@ -25,20 +25,23 @@ struct AttnParams {
   int* status;
 };
 
-// Tensor-core (bf16) split-KV attention partials; key splits must be multiples of 64.
-cudaError_t launch_attn_mma(const AttnParams& p, cudaStream_t st);
+// Tensor-core (bf16) attention: the n_splits CTAs of one (request, KV head) form a
+// cluster and merge through distributed shared memory into out [R, n_q*d] (bf16).
+// kps must be a multiple of 64 and n_splits <= kMaxAttnCluster.
+constexpr int kMaxAttnCluster = 16;
+cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st, bool pdl);
 
-// Split-KV attention partials, then the log-sum-exp merge into out [R, n_q*d].
-cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st);
+// CUDA-core split-KV attention partials (fp32 path), then the log-sum-exp merge into out [R, n_q*d].
+cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st, bool pdl);
 
 // x[m] = E[token(m)] (token = anchor for block index 0, mask id otherwise), h[m] = RMSNorm(x[m]) * gain.
-void launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
-                       int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
-                       cudaStream_t st);
+cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
+                              int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
+                              cudaStream_t st, bool pdl);
 // h[m] = RMSNorm(x[m]) * gain; optional fp32 copy of h into y.
-void launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
-                    cudaStream_t st);
+cudaError_t launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
+                           cudaStream_t st, bool pdl);
 // draft[b, i-1] = index(keys[b*B + i]) for i >= 1; every key reset to 0.
-void launch_argmax_finalize(unsigned long long* keys, int bs, int B, int* draft, cudaStream_t st);
+cudaError_t launch_argmax_finalize(unsigned long long* keys, int bs, int B, int* draft, cudaStream_t st, bool pdl);
 
 }  // namespace dfl

@@ -72,6 +72,8 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const ET* embe
                                                                   int B, int V, int H, const float* gain,
                                                                   float eps, float* x, HT* h, int* status) {
   __shared__ float red[32];
+  grid_dep_wait();
+  grid_dep_launch();
   const int m = blockIdx.x;
   int tok = (m % B) == 0 ? anchor[m / B] : mask_id;
   if (tok < 0 || tok >= V) {
@@ -102,6 +104,8 @@ template <int VPT, typename HT>
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* x, int H, const float* gain, float eps,
                                                                HT* h, float* y) {
   __shared__ float red[32];
+  grid_dep_wait();
+  grid_dep_launch();
   const int m = blockIdx.x;
   float4 v[VPT];
   const float ss = load_row<VPT>(x + (size_t)m * H, H, v);
@@ -109,6 +113,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* x, i
 }
 
 __global__ void argmax_finalize_kernel(unsigned long long* keys, int bs, int B, int* draft) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= bs * B) return;
   const int b = e / B, i = e % B;
@@ -118,54 +124,59 @@ __global__ void argmax_finalize_kernel(unsigned long long* keys, int bs, int B, 
 }
 
 template <int VPT>
-static void embed_norm_vpt(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
-                           int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
-                           cudaStream_t st) {
+static cudaError_t embed_norm_vpt(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R,
+                                  int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16,
+                                  int* status, cudaStream_t st, bool pdl) {
+  const dim3 g(R), b(kNormThreads);
   if (embed_bf16 && h_bf16)
-    embed_norm_kernel<VPT, __nv_bfloat16, __nv_bfloat16><<<R, kNormThreads, 0, st>>>(
-        (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, status);
-  else if (!embed_bf16 && !h_bf16)
-    embed_norm_kernel<VPT, float, float><<<R, kNormThreads, 0, st>>>((const float*)embed, anchor, mask_id, B, V, H,
-                                                                     gain, eps, x, (float*)h, status);
-  else if (embed_bf16)
-    embed_norm_kernel<VPT, __nv_bfloat16, float><<<R, kNormThreads, 0, st>>>(
-        (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (float*)h, status);
-  else
-    embed_norm_kernel<VPT, float, __nv_bfloat16><<<R, kNormThreads, 0, st>>>(
-        (const float*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, status);
+    return launch_kernel(embed_norm_kernel<VPT, __nv_bfloat16, __nv_bfloat16>, g, b, 0, st, pdl,
+                         (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h,
+                         status);
+  if (!embed_bf16 && !h_bf16)
+    return launch_kernel(embed_norm_kernel<VPT, float, float>, g, b, 0, st, pdl, (const float*)embed, anchor,
+                         mask_id, B, V, H, gain, eps, x, (float*)h, status);
+  if (embed_bf16)
+    return launch_kernel(embed_norm_kernel<VPT, __nv_bfloat16, float>, g, b, 0, st, pdl,
+                         (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (float*)h, status);
+  return launch_kernel(embed_norm_kernel<VPT, float, __nv_bfloat16>, g, b, 0, st, pdl, (const float*)embed, anchor,
+                       mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, status);
 }
 
-void launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
-                       int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
-                       cudaStream_t st) {
+cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
+                              int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
+                              cudaStream_t st, bool pdl) {
   const int vpt = (H / 4 + kNormThreads - 1) / kNormThreads;
-  if (vpt <= 1) embed_norm_vpt<1>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st);
-  else if (vpt <= 2) embed_norm_vpt<2>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st);
-  else if (vpt <= 4) embed_norm_vpt<4>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st);
-  else embed_norm_vpt<8>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st);
+  if (vpt <= 1)
+    return embed_norm_vpt<1>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st, pdl);
+  if (vpt <= 2)
+    return embed_norm_vpt<2>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st, pdl);
+  if (vpt <= 4)
+    return embed_norm_vpt<4>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st, pdl);
+  return embed_norm_vpt<8>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st, pdl);
 }
 
 template <int VPT>
-static void rmsnorm_vpt(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
-                        cudaStream_t st) {
+static cudaError_t rmsnorm_vpt(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16,
+                               float* y, cudaStream_t st, bool pdl) {
   if (h_bf16)
-    rmsnorm_kernel<VPT, __nv_bfloat16><<<R, kNormThreads, 0, st>>>(x, H, gain, eps, (__nv_bfloat16*)h, y);
-  else
-    rmsnorm_kernel<VPT, float><<<R, kNormThreads, 0, st>>>(x, H, gain, eps, (float*)h, y);
+    return launch_kernel(rmsnorm_kernel<VPT, __nv_bfloat16>, dim3(R), dim3(kNormThreads), 0, st, pdl, x, H, gain,
+                         eps, (__nv_bfloat16*)h, y);
+  return launch_kernel(rmsnorm_kernel<VPT, float>, dim3(R), dim3(kNormThreads), 0, st, pdl, x, H, gain, eps,
+                       (float*)h, y);
 }
 
-void launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
-                    cudaStream_t st) {
+cudaError_t launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
+                           cudaStream_t st, bool pdl) {
   const int vpt = (H / 4 + kNormThreads - 1) / kNormThreads;
-  if (vpt <= 1) rmsnorm_vpt<1>(x, R, H, gain, eps, h, h_bf16, y, st);
-  else if (vpt <= 2) rmsnorm_vpt<2>(x, R, H, gain, eps, h, h_bf16, y, st);
-  else if (vpt <= 4) rmsnorm_vpt<4>(x, R, H, gain, eps, h, h_bf16, y, st);
-  else rmsnorm_vpt<8>(x, R, H, gain, eps, h, h_bf16, y, st);
+  if (vpt <= 1) return rmsnorm_vpt<1>(x, R, H, gain, eps, h, h_bf16, y, st, pdl);
+  if (vpt <= 2) return rmsnorm_vpt<2>(x, R, H, gain, eps, h, h_bf16, y, st, pdl);
+  if (vpt <= 4) return rmsnorm_vpt<4>(x, R, H, gain, eps, h, h_bf16, y, st, pdl);
+  return rmsnorm_vpt<8>(x, R, H, gain, eps, h, h_bf16, y, st, pdl);
 }
 
-void launch_argmax_finalize(unsigned long long* keys, int bs, int B, int* draft, cudaStream_t st) {
+cudaError_t launch_argmax_finalize(unsigned long long* keys, int bs, int B, int* draft, cudaStream_t st, bool pdl) {
   const int n = bs * B;
-  argmax_finalize_kernel<<<(n + 255) / 256, 256, 0, st>>>(keys, bs, B, draft);
+  return launch_kernel(argmax_finalize_kernel, dim3((n + 255) / 256), dim3(256), 0, st, pdl, keys, bs, B, draft);
 }
 
 }  // namespace dfl

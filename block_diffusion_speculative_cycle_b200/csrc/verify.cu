@@ -7,6 +7,7 @@
 // draft[i-1] against argmax row i-1, next = argmax row a; it then zeroes the
 // request's keys and ticket so the workspace is ready for the next call.
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/dflash.h"
@@ -81,6 +82,8 @@ __global__ void __launch_bounds__(kVerifyThreads) verify_kernel(const T* logits,
                                                                  unsigned long long* keys, int* tickets,
                                                                  int* accepted, int* next_token) {
   __shared__ unsigned long long red[kVerifyThreads / 32];
+  grid_dep_wait();
+  grid_dep_launch();
   const int c = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
   const T* row = logits + ((size_t)b * B + j) * V;
   const int v0 = c * kVerifyChunk, v1 = min(V, v0 + kVerifyChunk);
@@ -107,6 +110,23 @@ __global__ void __launch_bounds__(kVerifyThreads) verify_kernel(const T* logits,
   }
 }
 
+// Programmatic dependent launch for verify (on unless DFLASH_PDL=0).
+static bool verify_pdl() {
+  static const bool on = [] {
+    const char* e = std::getenv("DFLASH_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+template <typename T>
+static cudaError_t launch_verify(const T* logits, const int* draft, int bs, int B, int V, unsigned long long* keys,
+                                 int* tickets, int* accepted, int* next_token, cudaStream_t st) {
+  const dim3 grid((unsigned)((V + kVerifyChunk - 1) / kVerifyChunk), (unsigned)B, (unsigned)bs);
+  return launch_kernel(verify_kernel<T>, grid, dim3(kVerifyThreads), 0, st, verify_pdl(), logits, draft, B, V, keys,
+                       tickets, accepted, next_token);
+}
+
 }  // namespace dfl
 
 extern "C" size_t dflash_verify_workspace_size(int bs, int B) {
@@ -126,15 +146,13 @@ extern "C" dflash_status dflash_verify(const void* d_logits, dflash_dtype logits
   if (bs > 65535 || B > 65535) return DFLASH_ERR_UNSUPPORTED;
   auto* keys = reinterpret_cast<unsigned long long*>(d_workspace);
   auto* tickets = reinterpret_cast<int*>(reinterpret_cast<char*>(d_workspace) + (size_t)bs * B * 8);
-  const dim3 grid((unsigned)((V + dfl::kVerifyChunk - 1) / dfl::kVerifyChunk), (unsigned)B, (unsigned)bs);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (logits_dtype == DFLASH_BF16)
-    dfl::verify_kernel<__nv_bfloat16><<<grid, dfl::kVerifyThreads, 0, st>>>(
-        (const __nv_bfloat16*)d_logits, d_draft, B, V, keys, tickets, d_accepted, d_next_token);
-  else
-    dfl::verify_kernel<float><<<grid, dfl::kVerifyThreads, 0, st>>>((const float*)d_logits, d_draft, B, V, keys,
-                                                                    tickets, d_accepted, d_next_token);
-  return cudaGetLastError() == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
+  const cudaError_t e =
+      logits_dtype == DFLASH_BF16
+          ? dfl::launch_verify((const __nv_bfloat16*)d_logits, d_draft, bs, B, V, keys, tickets, d_accepted,
+                               d_next_token, st)
+          : dfl::launch_verify((const float*)d_logits, d_draft, bs, B, V, keys, tickets, d_accepted, d_next_token, st);
+  return e == cudaSuccess ? DFLASH_OK : DFLASH_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- no-allocation variant
