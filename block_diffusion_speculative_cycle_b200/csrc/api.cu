@@ -55,6 +55,9 @@ struct dflash_ctx {
   bool bf16 = false;
   bool force_simt = false;
   bool use_pdl = false;
+  bool debug = false;
+  int force_splits = 0;   // DFLASH_SPLITS: fixed K-split count (experiments)
+  int force_stages = 0;   // DFLASH_STAGES: fixed ring depth (experiments)
   int num_sms = 148;
   const void* fc = nullptr;
   const void* embed = nullptr;
@@ -79,11 +82,12 @@ struct dflash_ctx {
   float* att_l = nullptr;
   size_t att_rows = 0;   // capacity in (split, row) pairs
   int* status = nullptr;
+  double* inv_freq = nullptr;   // [head_dim/2] RoPE inverse frequencies
+  float* sumsq[2] = {nullptr, nullptr};   // deferred-norm partial sums of squares [H/128][rows], ping-pong
   EncodeTiledFn encode = nullptr;
   bool prof = false;
   std::vector<ProfRec> recs;
   std::map<std::tuple<const void*, long long, long long, long long, int>, CUtensorMap> maps;
-  std::map<std::pair<int, int>, int> cluster_cap;   // (m_tile*16 + stages, splits) -> co-resident clusters
 };
 
 namespace {
@@ -155,23 +159,14 @@ struct GemmSpec {
   EpiParams epi{};
 };
 
-// K splits per output tile (= cluster size): the largest split count whose
-// grid still fits on the GPU in one wave (every CTA co-resident), so the weight
-// stream runs on as many SMs as possible without a tail wave.
-int choose_splits(dflash_ctx* ctx, int units, int num_kb, int m_tile, int stages) {
-  for (int s = kMaxClusterSplits; s >= 2; --s) {
-    if (num_kb / s < 2) continue;
-    const auto key = std::make_pair(m_tile * 16 + stages, s);
-    auto it = ctx->cluster_cap.find(key);
-    int cap;
-    if (it != ctx->cluster_cap.end()) {
-      cap = it->second;
-    } else {
-      cap = gemm_tc_max_active_clusters(m_tile, stages, s);
-      ctx->cluster_cap[key] = cap;
-    }
-    if (units <= cap) return s;
-  }
+// K splits per output tile (= cluster size): the largest count (<= 8) that keeps
+// the grid within two CTAs per SM, so every CTA streams from the start and a
+// third slot per SM stays free for the next kernel's CTAs to start and prefetch
+// their weights (programmatic dependent launch).
+int choose_splits(dflash_ctx* ctx, int units, int num_kb) {
+  const int slots = 2 * ctx->num_sms;
+  for (int s = kMaxClusterSplits; s >= 2; --s)
+    if (num_kb / s >= 2 && units * s <= slots) return s;
   return 1;
 }
 
@@ -237,16 +232,28 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   p.num_kb = g.K / 64;
   p.n_tiles = n_tiles;
   const int units = n_tiles * p.m_blocks;
-  const int per_sm = p.m_tile <= 64 ? 2 : 1;
-  const size_t budget = per_sm == 2 ? 110 * 1024 : 220 * 1024;
+  p.splits = ctx->force_splits > 0 ? std::min(ctx->force_splits, std::max(1, p.num_kb / 2))
+                                   : choose_splits(ctx, units, p.num_kb);
+  // ring depth: while m_tile <= 32 keep each CTA (ring + receive buffer) within a
+  // third of the SM's shared memory, so three CTAs fit; otherwise use what fits.
+  // The split epilogue reuses the ring for this split's rows (m_tile x 128 fp32)
+  // plus one chunk; if that does not fit, use fewer splits.
   const int sb = kTileN * 64 * 2 + p.m_tile * 128;
-  p.stages = (int)std::min<size_t>(8, (budget - 1024) / sb);
-  if (p.stages < 2) return DFLASH_ERR_UNSUPPORTED;
-  p.splits = choose_splits(ctx, units, p.num_kb, p.m_tile, p.stages);
+  const size_t budget = p.m_tile <= 32 ? 74 * 1024 : (p.m_tile <= 64 ? 110 * 1024 : 220 * 1024);
+  const size_t chunk_bytes = (size_t)kChunkRows * kChunkLd * 4;
+  for (;;) {
+    const size_t fixed = gemm_tc_smem_bytes(p.m_tile, 0, p.splits);
+    p.stages = budget > fixed ? (int)std::min<size_t>(8, (budget - fixed) / sb) : 0;
+    if (ctx->force_stages >= 2 && fixed + (size_t)ctx->force_stages * sb <= 225 * 1024) p.stages = ctx->force_stages;
+    const size_t need = (p.splits > 1 ? (size_t)p.m_tile * kTileN * 4 : 0) + chunk_bytes;
+    if (p.stages >= 2 && (size_t)p.stages * sb >= need) break;
+    if (p.splits == 1) return DFLASH_ERR_UNSUPPORTED;
+    p.splits = p.splits > 2 ? p.splits / 2 : 1;
+  }
   p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
-  // the cluster reduction stages m_tile x 128 fp32 plus one epilogue chunk in the ring's memory
-  if (p.splits > 1 && (size_t)p.stages * sb < (size_t)p.m_tile * kTileN * 4 + kChunkRows * kChunkLd * 4)
-    return DFLASH_ERR_UNSUPPORTED;
+  if (ctx->debug)
+    std::fprintf(stderr, "dflash gemm tag=%d M=%d K=%d tiles=%d m_tile=%d stages=%d splits=%d\n", g.tag, g.M, g.K,
+                 n_tiles, p.m_tile, p.stages, p.splits);
   p.use_pdl = ctx->use_pdl ? 1 : 0;
   const int box_w = g.paired ? kTileN / 2 : kTileN;
   const int nmaps = g.paired ? 2 : g.n_seg;
@@ -254,6 +261,16 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
     if (!get_map(ctx, g.w[s], g.seg_rows[s], g.K, g.K, box_w, &p.wmap[s])) return DFLASH_ERR_CUDA;
   if (!get_map(ctx, g.x, g.M, g.K, g.ldx, p.m_tile, &p.xmap)) return DFLASH_ERR_CUDA;
   return cuda_status(launch_gemm_tc(p, st), "gemm_tc launch");
+}
+
+// The GEMM's input rows are x ⊙ gain; scale its accumulators by the row's rstd
+// from the partial sums of squares the previous residual GEMM left in `part`.
+void set_deferred_norm(dflash_ctx* ctx, EpiParams& e, const float* part, int rows) {
+  e.norm_part = part;
+  e.n_part = ctx->cfg.hidden / kTileN;
+  e.ld_part = rows;
+  e.norm_inv_h = 1.0f / (float)ctx->cfg.hidden;
+  e.norm_eps = ctx->cfg.rms_eps;
 }
 
 #define DFL_CHECK(call)                       \
@@ -306,6 +323,14 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   ctx->bf16 = c.dtype == DFLASH_BF16;
   const char* env = std::getenv("DFLASH_FORCE_SIMT");
   ctx->force_simt = env && env[0] == '1';
+  env = std::getenv("DFLASH_DEBUG");
+  ctx->debug = env && env[0] == '1';
+  env = std::getenv("DFLASH_SPLITS");
+  ctx->force_splits = env ? std::atoi(env) : 0;
+  if (ctx->force_splits > kMaxClusterSplits) ctx->force_splits = kMaxClusterSplits;
+  env = std::getenv("DFLASH_STAGES");
+  ctx->force_stages = env ? std::atoi(env) : 0;
+  if (ctx->force_stages > 8) ctx->force_stages = 8;
   env = std::getenv("DFLASH_PDL");
   ctx->use_pdl = !(env && env[0] == '0');
   int dev = 0;
@@ -367,6 +392,9 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   const size_t o_attm = take(ctx->att_rows * 4);
   const size_t o_attl = take(ctx->att_rows * 4);
   const size_t o_st = take(256);
+  const size_t o_freq = take((size_t)c.head_dim / 2 * sizeof(double));
+  const size_t o_ss0 = take((size_t)(c.hidden / 128) * R * 4);
+  const size_t o_ss1 = take((size_t)(c.hidden / 128) * R * 4);
   ctx->ws_bytes = off;
   if (cudaMalloc(&ctx->ws, off) != cudaSuccess) {
     cudaGetLastError();
@@ -392,6 +420,19 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   ctx->att_m = (float*)(b + o_attm);
   ctx->att_l = (float*)(b + o_attl);
   ctx->status = (int*)(b + o_st);
+  ctx->inv_freq = (double*)(b + o_freq);
+  ctx->sumsq[0] = (float*)(b + o_ss0);
+  ctx->sumsq[1] = (float*)(b + o_ss1);
+  {
+    // theta^(-2i/d), i = 0..d/2-1, in double
+    std::vector<double> f(c.head_dim / 2);
+    for (int i = 0; i < c.head_dim / 2; ++i) f[i] = std::pow((double)c.rope_theta, -2.0 * i / c.head_dim);
+    if (cudaMemcpy(ctx->inv_freq, f.data(), f.size() * sizeof(double), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(ctx->ws);
+      delete ctx;
+      return DFLASH_ERR_CUDA;
+    }
+  }
   *out = ctx;
   return DFLASH_OK;
 }
@@ -504,7 +545,7 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
       e.rope_mask |= 1u << (2 * i);
     }
     e.head_dim = c.head_dim;
-    e.log2_theta = std::log2((double)c.rope_theta);
+    e.inv_freq = ctx->inv_freq;
     e.rows_per_req = max_new;
     e.pos_base = d_start_pos;
     e.row_count = d_n_new;
@@ -584,9 +625,10 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     qkv.epi.ld_out[2] = KVD;
     qkv.epi.rope_mask = 3u;
     qkv.epi.head_dim = c.head_dim;
-    qkv.epi.log2_theta = std::log2((double)c.rope_theta);
+    qkv.epi.inv_freq = ctx->inv_freq;
     qkv.epi.rows_per_req = B;
     qkv.epi.pos_base = d_ctx_len;
+    if (l > 0) set_deferred_norm(ctx, qkv.epi, ctx->sumsq[1], R);   // rows carry the previous layer's norm
     DFL_CHECK(run_gemm(ctx, qkv, st));
 
     AttnParams ap{};
@@ -634,14 +676,12 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     o.epi.kind = EPI_RESID;
     o.epi.x = ctx->x;
     o.epi.ldx = H;
+    // the MLP norm is deferred: x ⊙ gain now, the row scales in the gate/up epilogue
+    o.epi.gamma_next = ctx->mlp_norm[l];
+    o.epi.xg = ctx->h;
+    o.epi.sumsq = ctx->sumsq[0];
+    o.epi.ld_part = R;
     DFL_CHECK(run_gemm(ctx, o, st));
-
-    {
-      ProfScope prof(ctx, PK_RMSNORM, st, norm_bytes, 0);
-      DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->mlp_norm[l], c.rms_eps, ctx->h, hb, nullptr, st,
-                                           ctx->use_pdl),
-                            "rmsnorm launch"));
-    }
 
     GemmSpec gu;
     gu.x = ctx->h;
@@ -657,6 +697,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     gu.epi.kind = EPI_SWIGLU;
     gu.epi.out[0] = ctx->act;
     gu.epi.ld_out[0] = c.intermediate;
+    set_deferred_norm(ctx, gu.epi, ctx->sumsq[0], R);
     DFL_CHECK(run_gemm(ctx, gu, st));
 
     GemmSpec dn;
@@ -671,6 +712,12 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     dn.epi.kind = EPI_RESID;
     dn.epi.x = ctx->x;
     dn.epi.ldx = H;
+    // the next layer's attention norm (or the final norm) is deferred the same way
+    const bool last = l + 1 == c.n_layers;
+    dn.epi.gamma_next = last ? ctx->final_norm : ctx->attn_norm[l + 1];
+    dn.epi.xg = ctx->h;
+    dn.epi.sumsq = ctx->sumsq[1];
+    dn.epi.ld_part = R;
     DFL_CHECK(run_gemm(ctx, dn, st));
 
     if (d_hidden_out) {
@@ -678,15 +725,13 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
       if (cudaMemcpyAsync(d_hidden_out + l * layer_stride, ctx->x, layer_stride * 4, cudaMemcpyDeviceToDevice,
                           st) != cudaSuccess)
         return DFLASH_ERR_CUDA;
-    }
-    const bool last = l + 1 == c.n_layers;
-    {
-      ProfScope prof(ctx, PK_RMSNORM, st, norm_bytes, 0);
-      DFL_CHECK(cuda_status(
-          launch_rmsnorm(ctx->x, R, H, last ? ctx->final_norm : ctx->attn_norm[l + 1], c.rms_eps, ctx->h, hb,
-                         last && d_hidden_out ? d_hidden_out + (size_t)c.n_layers * layer_stride : nullptr, st,
-                         ctx->use_pdl),
-          "rmsnorm launch"));
+      if (last) {
+        // the final normed rows, for parity checks only (the LM head uses the deferred form)
+        ProfScope prof2(ctx, PK_RMSNORM, st, norm_bytes, 0);
+        DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, nullptr, hb,
+                                             d_hidden_out + (size_t)c.n_layers * layer_stride, st, ctx->use_pdl),
+                              "rmsnorm launch"));
+      }
     }
   }
   if (c.n_layers == 0 && d_hidden_out)
@@ -705,6 +750,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   lm.tag = TAG_LM;
   lm.epi.kind = EPI_ARGMAX;
   lm.epi.keys = ctx->keys;
+  if (c.n_layers > 0) set_deferred_norm(ctx, lm.epi, ctx->sumsq[1], R);
   DFL_CHECK(run_gemm(ctx, lm, st));
   {
     ProfScope prof(ctx, PK_ARGMAX, st, (double)R * 8 * 2 + (double)bs * (B - 1) * 4, 0);

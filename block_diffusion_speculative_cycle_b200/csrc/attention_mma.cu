@@ -9,14 +9,13 @@
 // from the request's cache pages, the B block keys from the block K/V rows.
 // Per tile: S = Q·Kᵀ (m16n8k16), online softmax in fp32 (exp2 domain, quad
 // shuffles), O += P·V with P re-packed from the S accumulators. The split's
-// state (unnormalised O, running max m, sum l) is staged in shared memory; after a
-// cluster barrier each CTA combines a share of the rows over all splits through
-// distributed shared memory (log-sum-exp weights, split order) and writes them.
-#include <cooperative_groups.h>
-
+// state (unnormalised O, running max m, sum l) is staged per row and each block
+// of rows is bulk-copied into the receive buffer of the cluster CTA that owns
+// those rows (distributed shared memory, counted on that CTA's mbarrier); each
+// owner waits for exactly its rows, combines the splits (log-sum-exp weights,
+// split order) and writes them.
 #include "kernels.cuh"
-
-namespace cg = cooperative_groups;
+#include "sm100.cuh"
 
 namespace dfl {
 
@@ -24,9 +23,8 @@ namespace {
 
 constexpr int kKT = 64;   // keys per tile
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
+using sm100::smem_addr;
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return smem_addr(p); }
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                : "memory");
@@ -67,18 +65,26 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 
 }  // namespace
 
-// Stages of the K/V ring: 3 for up to 64 query rows, 2 for 128 (both fit two CTAs per SM).
-template <int D, int NST>
+// Stages of the K/V ring: 3 for up to 64 query rows, 2 for 128. KS warp groups
+// split every 64-key tile (KS = 2: group g takes keys 32g .. 32g+31), each with
+// its own online-softmax state, merged in shared memory after the loop.
+template <int D, int NST, int KS>
 __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, __nv_bfloat16* out) {
-  constexpr int CH = D / 8;    // 16-byte chunks per row
+  constexpr int CH = D / 8;          // 16-byte chunks per row
+  constexpr int REC = D + 4;         // merge record: O (D floats), m, l, two pad words (16-byte multiple)
+  constexpr int NT = kKT / 8 / KS;   // score n-tiles of 8 keys per warp group
+  constexpr int KK = kKT / 16 / KS;  // P·V k-steps of 16 keys per warp group
   extern __shared__ __align__(128) uint8_t smem_raw[];
+  __shared__ uint64_t recv_bar;
   const int nr = p.g * p.B;
   const int rows_pad = ((nr + 15) / 16) * 16;
+  const int slices = rows_pad / 16;
   __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem_raw);   // [rows_pad][D]
   __nv_bfloat16* ring = qs + rows_pad * D;                           // NST x ([kKT][D] K, [kKT][D] V)
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const int grp = warp / slices, slice = warp % slices;
   const int gid = lane >> 2, tig = lane & 3;
   const int q_dim = p.n_q * D, kv_dim = p.n_kv * D;
   const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q);
@@ -86,8 +92,11 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
   const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(p.vblk);
   const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(p.kc);
   const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(p.vc);
-  grid_dep_wait();
-  grid_dep_launch();
+  // The context K/V were written by the injection kernels, which completed
+  // before this kernel could be launched (each kernel of the chain waits for its
+  // predecessor before it lets its successor start), and ctx_len / the page
+  // table come from the caller. So the context tiles are fetched before the
+  // wait; q and the block K/V come from the immediately preceding kernel.
 
   int P = p.ctx_len[b];
   if (P < 0 || P > p.max_ctx) {
@@ -98,9 +107,37 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
   const int k0 = s * p.kps, k1 = min(T_all, k0 + p.kps);
   const int n_tiles = k1 > k0 ? (k1 - k0 + kKT - 1) / kKT : 0;
 
+  const int S = p.n_splits;
+  const int per = (nr + S - 1) / S;                       // merged rows owned by each split
+  const int own_lo = min(nr, s * per), own_hi = min(nr, own_lo + per);
+  if (S > 1 && tid == 0) {
+    sm100::mbar_init(&recv_bar, 1);
+    sm100::fence_mbar_init();
+    sm100::mbar_arrive_expect_tx(&recv_bar, (uint32_t)(S * (own_hi - own_lo) * REC * 4));
+  }
+
+  // Tiles start at multiples of 64 keys (kps is a multiple of 64). When a tile
+  // holds only context keys and the page size is a multiple of 64, its 64 keys
+  // are one contiguous block of one page: resolve that page once.
+  const bool page_tiles = (p.page_size % kKT) == 0;
+  auto context_tile = [&](int kt) { return page_tiles && kt + kKT <= min(P, k1); };
   auto load_tile = [&](int kt, int stage) {
     __nv_bfloat16* kd = ring + stage * 2 * kKT * D;
     __nv_bfloat16* vd = kd + kKT * D;
+    if (context_tile(kt)) {
+      const int slot = kt / p.page_size;
+      const int page = slot < p.max_pages ? __ldg(p.page_table + (size_t)b * p.max_pages + slot) : -1;
+      const bool ok = page >= 0 && page < p.num_pages;
+      if (!ok && tid == 0) flag_error(p.status, ST_BAD_PAGE);
+      const size_t base = ok ? (((size_t)page * p.n_kv + h) * p.page_size + kt % p.page_size) * D : 0;
+      for (int e = tid; e < kKT * CH; e += nthr) {
+        const int r = e / CH, c = e % CH;
+        const size_t off = base + (size_t)r * D + c * 8;
+        cp_async16(kd + swz<D>(r, c), ok ? kc + off : kc, ok ? 16 : 0);
+        cp_async16(vd + swz<D>(r, c), ok ? vc + off : vc, ok ? 16 : 0);
+      }
+      return;
+    }
     for (int e = tid; e < kKT * CH; e += nthr) {
       const int r = e / CH, c = e % CH, key = kt + r;
       const __nv_bfloat16* ksrc = kb;
@@ -130,7 +167,14 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     }
   };
 
-  // group 0: Q rows (r = j*B + i: query head h*g + j, block row i) and tile 0; groups 1..NST-1: tiles 1..
+  // the first NST tiles: pure-context ones now, the rest (and Q) after the wait
+#pragma unroll
+  for (int i = 0; i < NST; ++i)
+    if (i < n_tiles && context_tile(k0 + i * kKT)) load_tile(k0 + i * kKT, i);
+  cp_async_commit();
+  grid_dep_wait();
+  grid_dep_launch();
+  // Q rows r = j*B + i: query head h*g + j, block row i
   for (int e = tid; e < rows_pad * CH; e += nthr) {
     const int r = e / CH, c = e % CH;
     const __nv_bfloat16* src = q;
@@ -143,50 +187,56 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     cp_async16(qs + swz<D>(r, c), src, bytes);
   }
 #pragma unroll
-  for (int i = 0; i < NST; ++i) {
-    if (i < n_tiles) load_tile(k0 + i * kKT, i);
-    cp_async_commit();
-  }
+  for (int i = 0; i < NST; ++i)
+    if (i < n_tiles && !context_tile(k0 + i * kKT)) load_tile(k0 + i * kKT, i);
+  cp_async_commit();
 
-  const bool active = warp * 16 < nr;
+  const bool active = slice * 16 < nr;
   uint32_t qf[D / 16][4];
   const float sl2 = p.scale * 1.4426950408889634f;   // softmax in the exp2 domain
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows gid, gid+8 of this warp
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows gid, gid+8 of this slice
   float o[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 
   for (int t = 0; t < n_tiles; ++t) {
-    cp_async_wait<NST - 1>();   // tile t (and Q) have landed
+    // tiles < NST (and Q) landed with the two prologue groups; tile t >= NST with
+    // the group committed NST iterations ago (one group per iteration)
+    if (t == 0)
+      cp_async_wait<0>();
+    else
+      cp_async_wait<NST - 1>();
     __syncthreads();
     if (active) {
       if (t == 0) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int mat = lane >> 3, r = lane & 7;
-          ldsm_x4(qf[kk], qs + swz<D>(warp * 16 + r + 8 * (mat & 1), 2 * kk + (mat >> 1)));
+          ldsm_x4(qf[kk], qs + swz<D>(slice * 16 + r + 8 * (mat & 1), 2 * kk + (mat >> 1)));
         }
       }
-      const int kt = k0 + t * kKT;
-      const __nv_bfloat16* kt_s = ring + (t % NST) * 2 * kKT * D;
-      const __nv_bfloat16* vt_s = kt_s + kKT * D;
-      float sc[kKT / 8][4];
+      const int kt = k0 + t * kKT + grp * (kKT / KS);   // this group's first key
+      const __nv_bfloat16* kt_s = ring + (t % NST) * 2 * kKT * D + grp * (kKT / KS) * D;
+      const __nv_bfloat16* vt_s = ring + (t % NST) * 2 * kKT * D + kKT * D + grp * (kKT / KS) * D;
+      float sc[NT][4];
 #pragma unroll
-      for (int n = 0; n < kKT / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+      for (int n = 0; n < NT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
 #pragma unroll
-        for (int n = 0; n < kKT / 8; n += 2) {
+        for (int n = 0; n < NT; n += 2) {
           const int mat = lane >> 3, r = lane & 7;
+          const int kr = grp * (kKT / KS) + n * 8 + r + 8 * (mat >> 1);   // key row within the tile
           uint32_t bfr[4];
-          ldsm_x4(bfr, kt_s + swz<D>(n * 8 + r + 8 * (mat >> 1), 2 * kk + (mat & 1)));
+          ldsm_x4(bfr, ring + (t % NST) * 2 * kKT * D + swz<D>(kr, 2 * kk + (mat & 1)));
           mma_16816(sc[n], qf[kk], bfr[0], bfr[1]);
           mma_16816(sc[n + 1], qf[kk], bfr[2], bfr[3]);
         }
       }
+      (void)kt_s;
       float mx0 = m0, mx1 = m1;
 #pragma unroll
-      for (int n = 0; n < kKT / 8; ++n) {
+      for (int n = 0; n < NT; ++n) {
         const int key = kt + n * 8 + 2 * tig;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -202,15 +252,18 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, m));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, m));
       }
-      const float a0 = exp2f(m0 - mx0), a1 = exp2f(m1 - mx1);
+      // a group whose keys are all masked keeps its state (-inf max) untouched
+      const float a0 = mx0 == -INFINITY ? 1.f : exp2f(m0 - mx0), a1 = mx1 == -INFINITY ? 1.f : exp2f(m1 - mx1);
       m0 = mx0;
       m1 = mx1;
       float rs0 = 0.f, rs1 = 0.f;
-      uint32_t pf[kKT / 16][4];
+      uint32_t pf[KK][4];
 #pragma unroll
-      for (int n = 0; n < kKT / 8; ++n) {
-        const float p00 = exp2f(sc[n][0] - m0), p01 = exp2f(sc[n][1] - m0);
-        const float p10 = exp2f(sc[n][2] - m1), p11 = exp2f(sc[n][3] - m1);
+      for (int n = 0; n < NT; ++n) {
+        const float p00 = mx0 == -INFINITY ? 0.f : exp2f(sc[n][0] - m0);
+        const float p01 = mx0 == -INFINITY ? 0.f : exp2f(sc[n][1] - m0);
+        const float p10 = mx1 == -INFINITY ? 0.f : exp2f(sc[n][2] - m1);
+        const float p11 = mx1 == -INFINITY ? 0.f : exp2f(sc[n][3] - m1);
         rs0 += p00 + p01;
         rs1 += p10 + p11;
         pf[n >> 1][(n & 1) * 2 + 0] = pack_bf16(p00, p01);
@@ -226,23 +279,28 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
         o[n][3] *= a1;
       }
 #pragma unroll
-      for (int kk = 0; kk < kKT / 16; ++kk) {
+      for (int kk = 0; kk < KK; ++kk) {
 #pragma unroll
         for (int n = 0; n < D / 8; n += 2) {
           const int mat = lane >> 3, r = lane & 7;
+          const int kr = grp * (kKT / KS) + kk * 16 + r + 8 * (mat & 1);
           uint32_t bfr[4];
-          ldsm_x4_t(bfr, vt_s + swz<D>(kk * 16 + r + 8 * (mat & 1), n + (mat >> 1)));
+          ldsm_x4_t(bfr, ring + (t % NST) * 2 * kKT * D + kKT * D + swz<D>(kr, n + (mat >> 1)));
           mma_16816(o[n], pf[kk], bfr[0], bfr[1]);
           mma_16816(o[n + 1], pf[kk], bfr[2], bfr[3]);
         }
       }
+      (void)vt_s;
     }
     __syncthreads();   // stage t % NST is free again
     if (t + NST < n_tiles) load_tile(k0 + (t + NST) * kKT, t % NST);
     cp_async_commit();
   }
   cp_async_wait<0>();
-  __syncthreads();   // every copy has landed and every warp is done with the ring
+  __syncthreads();   // every copy has landed and every warp is done with Q and the ring
+  // Past this barrier Q and the ring are dead; peers may write their merge records
+  // into the tail of this CTA's shared memory once every CTA of the cluster arrives.
+  if (S > 1) sm100::cluster_arrive_release();
 
   if (active) {
 #pragma unroll
@@ -251,11 +309,53 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
       l1 += __shfl_xor_sync(0xffffffffu, l1, m);
     }
   }
-  const int r0 = warp * 16 + gid, r1 = r0 + 8;
-  const int S = p.n_splits;
+  const int r0 = slice * 16 + gid, r1 = r0 + 8;
+  float* grp_area = reinterpret_cast<float*>(smem_raw);              // [rows_pad][REC] group-1 state
+  float* stg = grp_area + (KS > 1 ? (size_t)rows_pad * REC : 0);     // [nr][REC] this split's records
+  float* rcv = stg + (size_t)nr * REC;                               // [S][per][REC] received records
+  if (KS > 1) {
+    // fold the second warp group's (O, m, l) into the first group's registers
+    if (active && grp == 1) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float* rec = grp_area + (size_t)(half ? r1 : r0) * REC;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          const int d = n * 8 + 2 * tig;
+          *reinterpret_cast<float2*>(rec + d) = half ? make_float2(o[n][2], o[n][3]) : make_float2(o[n][0], o[n][1]);
+        }
+        if (tig == 0) {
+          rec[D] = half ? m1 : m0;
+          rec[D + 1] = half ? l1 : l0;
+        }
+      }
+    }
+    __syncthreads();
+    if (active && grp == 0) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const float* rec = grp_area + (size_t)(half ? r1 : r0) * REC;
+        const float mo = rec[D], lo_ = rec[D + 1];
+        float& mm = half ? m1 : m0;
+        float& ll = half ? l1 : l0;
+        const float M = fmaxf(mm, mo);
+        const float wa = mm == -INFINITY ? 0.f : exp2f(mm - M), wb = mo == -INFINITY ? 0.f : exp2f(mo - M);
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          const int d = n * 8 + 2 * tig;
+          const float2 ov = *reinterpret_cast<const float2*>(rec + d);
+          o[n][2 * half] = o[n][2 * half] * wa + ov.x * wb;
+          o[n][2 * half + 1] = o[n][2 * half + 1] * wa + ov.y * wb;
+        }
+        ll = ll * wa + lo_ * wb;
+        mm = M;
+      }
+    }
+  }
+  const bool writer = active && grp == 0;
   if (S == 1) {
     // the whole key range is here: normalise and write
-    if (active) {
+    if (writer) {
       const float i0 = 1.f / l0, i1 = 1.f / l1;
 #pragma unroll
       for (int n = 0; n < D / 8; ++n) {
@@ -275,46 +375,51 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     return;
   }
 
-  // ---- cluster merge: stage (O, m, l) of this split, then CTA `rank` combines its share of rows
-  float* so = reinterpret_cast<float*>(smem_raw);   // [nr][D] unnormalised O
-  float* sm = so + nr * D;                          // [nr] running max (exp2 domain)
-  float* sl = sm + nr;                              // [nr] running sum
-  if (active) {
+  // ---- cluster merge: stage this split's (O, m, l) records, bulk-copy each
+  // owner's block of rows into its receive buffer (counted on its barrier), then
+  // combine the rows this split owns over all splits, in split order.
+  if (writer) {
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      const int d = n * 8 + 2 * tig;
-      if (r0 < nr) *reinterpret_cast<float2*>(so + r0 * D + d) = make_float2(o[n][0], o[n][1]);
-      if (r1 < nr) *reinterpret_cast<float2*>(so + r1 * D + d) = make_float2(o[n][2], o[n][3]);
-    }
-    if (tig == 0) {
-      if (r0 < nr) {
-        sm[r0] = m0;
-        sl[r0] = l0;
-      }
-      if (r1 < nr) {
-        sm[r1] = m1;
-        sl[r1] = l1;
+    for (int half = 0; half < 2; ++half) {
+      const int r = half ? r1 : r0;
+      if (r < nr) {
+        float* rec = stg + (size_t)r * REC;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          const int d = n * 8 + 2 * tig;
+          *reinterpret_cast<float2*>(rec + d) = half ? make_float2(o[n][2], o[n][3]) : make_float2(o[n][0], o[n][1]);
+        }
+        if (tig == 0) {
+          rec[D] = half ? m1 : m0;
+          rec[D + 1] = half ? l1 : l0;
+        }
       }
     }
   }
-  cg::cluster_group cluster = cg::this_cluster();
-  cluster.sync();
-  const int per = (nr + S - 1) / S;
-  const int lo = s * per, hi = min(nr, lo + per);
-  const int nwarps = nthr >> 5;
-  for (int r = lo + warp; r < hi; r += nwarps) {
-    // lanes own splits for the max and the weights
-    float ms = -INFINITY, ls = 0.f;
-    if (lane < S) {
-      const float* rsm = cluster.map_shared_rank(sm, lane);
-      const float* rsl = cluster.map_shared_rank(sl, lane);
-      ms = rsm[r];
-      ls = rsl[r];
+  sm100::fence_proxy_async_smem();
+  __syncthreads();
+  sm100::cluster_wait_acquire();   // every CTA is past its loop and its receive barrier is set
+  if (tid == 0) {
+    const uint32_t rcv_s = smem_u32(rcv), bar_s = smem_u32(&recv_bar), stg_s = smem_u32(stg);
+    for (int k = 0; k < S; ++k) {
+      const int lo = min(nr, k * per), hi = min(nr, lo + per);
+      if (hi > lo)
+        sm100::bulk_copy_s2s(sm100::mapa_shared(rcv_s + (uint32_t)(s * per * REC * 4), (uint32_t)k),
+                             stg_s + (uint32_t)(lo * REC * 4), (uint32_t)((hi - lo) * REC * 4),
+                             sm100::mapa_shared(bar_s, (uint32_t)k));
     }
+    sm100::bulk_commit();
+  }
+  const bool got = sm100::mbar_wait(&recv_bar, 0, p.status);
+  const int nwarps = nthr >> 5;
+  for (int r = own_lo + warp; got && r < own_hi; r += nwarps) {
+    const int rl = r - own_lo;
+    const float ms = lane < S ? rcv[((size_t)lane * per + rl) * REC + D] : -INFINITY;
+    const float ls = lane < S ? rcv[((size_t)lane * per + rl) * REC + D + 1] : 0.f;
     float M = ms;
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-    const float w = lane < S ? exp2f(ms - M) : 0.f;
+    const float w = (lane < S && ms != -INFINITY) ? exp2f(ms - M) : 0.f;
     float L = ls * w;
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) L += __shfl_xor_sync(0xffffffffu, L, m);
@@ -324,37 +429,38 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
     for (int k = 0; k < S; ++k) {
       const float wk = __shfl_sync(0xffffffffu, w, k);
-      const float* ro = cluster.map_shared_rank(so, k) + r * D;
+      const float* src = rcv + ((size_t)k * per + rl) * REC;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(wk, ro[lane + 32 * c], acc[c]);
+      for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(wk, src[lane + 32 * c], acc[c]);
     }
     const int j = r / p.B, i = r % p.B;
     __nv_bfloat16* dst = out + (size_t)(b * p.B + i) * q_dim + (h * p.g + j) * D;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) dst[lane + 32 * c] = __float2bfloat16_rn(acc[c] * invL);
   }
-  cluster.sync();   // peers may still be reading this CTA's staging
+  if (tid == 0) sm100::bulk_wait_read_all();   // the staging has been read by every outgoing copy
 }
 
-static size_t attn_cluster_smem(int d, int rows_pad, int nst) {
+static size_t attn_cluster_smem(int d, int nr, int rows_pad, int nst, int ks, int splits) {
   const size_t loads = ((size_t)rows_pad + (size_t)nst * 2 * kKT) * d * 2;
-  const size_t merge = ((size_t)rows_pad * d + 2 * rows_pad) * 4;
+  const size_t per = (size_t)(nr + splits - 1) / splits;
+  const size_t rec = (size_t)(d + 4) * 4;
+  const size_t merge = (ks > 1 ? (size_t)rows_pad * rec : 0) + (splits > 1 ? (size_t)nr * rec + splits * per * rec : 0);
   return loads > merge ? loads : merge;
 }
 
-template <int D, int NST>
+template <int D, int NST, int KS>
 static cudaError_t launch_cluster_t(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {
   const int nr = p.g * p.B;
   const int rows_pad = ((nr + 15) / 16) * 16;
-  const int warps = rows_pad / 16;
-  const int threads = 32 * (warps < 4 ? 4 : warps);
-  const size_t smem = attn_cluster_smem(D, rows_pad, NST);
+  const int threads = 32 * KS * (rows_pad / 16);
+  const size_t smem = attn_cluster_smem(D, nr, rows_pad, NST, KS, p.n_splits);
   static size_t set = 0;
   if (smem > set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_cluster_kernel<D, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(attn_cluster_kernel<D, NST, KS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_cluster_kernel<D, NST>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(attn_cluster_kernel<D, NST, KS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     set = smem;
   }
@@ -372,14 +478,17 @@ static cudaError_t launch_cluster_t(const AttnParams& p, void* out, cudaStream_t
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.n_splits > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, attn_cluster_kernel<D, NST>, p, (__nv_bfloat16*)out);
+  return cudaLaunchKernelEx(&cfg, attn_cluster_kernel<D, NST, KS>, p, (__nv_bfloat16*)out);
 }
 
 cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {
   if (p.n_splits < 1 || p.n_splits > kMaxAttnCluster || p.kps % kKT) return cudaErrorInvalidValue;
+  // one warp per 16 query rows (one key group): two CTAs fit per SM by registers
+  // and shared memory, which keeps the clusters placeable all at once
   const bool wide = p.g * p.B > 64;
-  if (p.d == 128) return wide ? launch_cluster_t<128, 2>(p, out, st, pdl) : launch_cluster_t<128, 3>(p, out, st, pdl);
-  return wide ? launch_cluster_t<64, 2>(p, out, st, pdl) : launch_cluster_t<64, 3>(p, out, st, pdl);
+  if (p.d == 128)
+    return wide ? launch_cluster_t<128, 2, 1>(p, out, st, pdl) : launch_cluster_t<128, 3, 1>(p, out, st, pdl);
+  return wide ? launch_cluster_t<64, 2, 1>(p, out, st, pdl) : launch_cluster_t<64, 3, 1>(p, out, st, pdl);
 }
 
 }  // namespace dfl

@@ -85,16 +85,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // ---------------------------------------------------------------- RoPE
-// Rotate-half RoPE factor for pair index i (0 <= i < d/2) at position pos:
-// angle = pos * theta^(-2i/d), evaluated in double so that long contexts keep
-// full fp32 accuracy in cos/sin.
-__device__ __forceinline__ void rope_cos_sin(int pos, int i, int d, double log2_theta, float* c, float* s) {
-  double inv_freq = exp2(-2.0 * (double)i / (double)d * log2_theta);
-  double ang = (double)pos * inv_freq;
-  double sd, cd;
-  sincos(ang, &sd, &cd);
-  *c = (float)cd;
-  *s = (float)sd;
+// Rotate-half RoPE factors for a pair with inverse frequency inv_freq (double,
+// theta^(-2i/d)) at integer position pos. The angle pos*inv_freq is formed and
+// reduced to [-pi, pi] in double (one multiply, one rounding, one fma), so that
+// positions up to 2^24 keep full fp32 accuracy; cos/sin are then taken in fp32.
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
+  const double two_pi = 6.283185307179586;
+  const double a = (double)pos * inv_freq;
+  const double k = rint(a * (1.0 / two_pi));
+  const float r = (float)fma(-k, two_pi, a);
+  sincosf(r, s, c);
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }

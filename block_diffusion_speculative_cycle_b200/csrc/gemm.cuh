@@ -30,7 +30,7 @@ struct EpiParams {
   int ld_out[kMaxSeg];               // leading dimension (elements) of out[s] for STORE/QKV/SWIGLU
   unsigned int rope_mask;            // bit s: rotate segment s
   int head_dim;
-  double log2_theta;
+  const double* inv_freq;            // [head_dim/2] theta^(-2i/d), double
   int rows_per_req;                  // activation row m belongs to request m / rows_per_req
   const int* pos_base;               // [bs] absolute position of each request's first row
   const int* row_count;              // [bs] valid rows per request (nullptr: all)
@@ -38,6 +38,18 @@ struct EpiParams {
   int max_pages, num_pages, page_size, n_kv;
   float* x;                          // residual stream [M, ldx] fp32
   int ldx;
+  // Deferred RMSNorm of this GEMM's input rows (the input is x ⊙ gain, not yet
+  // normalised): acc *= rsqrt(sum_p norm_part[p * ld_part + row] / H + eps),
+  // the partial sums of squares summed in p order. Null: input already normalised.
+  const float* norm_part;
+  int n_part, ld_part;
+  float norm_inv_h, norm_eps;
+  // Residual epilogue extras: the next norm's operand xg = x_new ⊙ gamma_next
+  // (model dtype, [M, ldx]) and this tile's partial sums of squares of x_new,
+  // sumsq[tile * ld_part + row]. Null: not produced.
+  const float* gamma_next;
+  void* xg;
+  float* sumsq;
   unsigned long long* keys;          // [M] packed argmax keys
   int* status;
   int out_bf16;                      // 1: bf16 outputs, 0: fp32 outputs
@@ -56,10 +68,31 @@ __device__ __forceinline__ void store_out(void* base, size_t idx, float v, int b
     reinterpret_cast<float*>(base)[idx] = v;
 }
 
+// Scratch of the epilogue (shared memory, per CTA): row scales, then a 4 x 32 reduction area.
+constexpr int kEpiScratch = kChunkRows + 4 * kChunkRows;
+
+// Row scales of the deferred RMSNorm for rows row0 .. row0+nrows-1 into
+// scratch[0..nrows): threads t < nrows each sum their row's partials in order.
+// The caller synchronises the 128 threads before epilogue_chunk reads them.
+__device__ __forceinline__ void epilogue_row_scales(const EpiParams& e, int row0, int nrows, float* scratch, int t) {
+  if (!e.norm_part || t >= nrows) return;
+  float ss = 0.f;
+  for (int i = 0; i < e.n_part; ++i) ss += __ldcg(e.norm_part + (size_t)i * e.ld_part + row0 + t);
+  scratch[t] = rsqrtf(ss * e.norm_inv_h + e.norm_eps);
+}
+
 // Apply the epilogue to one staged chunk: acc[j * kChunkLd + t] holds the
-// accumulator of activation row row0 + j (j < nrows) and tile row t (0..127).
-// Called by 128 threads with t = their tile row; no barrier inside.
-__device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t) {
+// accumulator of activation row row0 + j (j < nrows) and tile row t (0..127),
+// scaled by scratch[j] when the input rows carry a deferred norm. Called by 128
+// threads with t = their tile row. The residual epilogue synchronises the 128
+// threads once (named barrier 2) when it produces partial sums of squares.
+__device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t,
+                                      float* scratch) {
+  const float* rs = e.norm_part ? scratch : nullptr;
+  auto A = [&](int j, int c) -> float {
+    const float v = acc[j * kChunkLd + c];
+    return rs ? v * rs[j] : v;
+  };
   switch (e.kind) {
     case EPI_STORE:
     case EPI_QKV: {
@@ -69,15 +102,16 @@ __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, in
       const int d = e.head_dim, half = d >> 1;
       const int jd = n % d;
       const int tp = jd < half ? t + half : t - half;
+      const double f = rope ? __ldg(e.inv_freq + jd % half) : 0.0;
       for (int j = 0; j < nrows; ++j) {
         const int m = row0 + j;
-        float v = acc[j * kChunkLd + t];
+        float v = A(j, t);
         if (rope) {
           const int req = m / e.rows_per_req, i = m % e.rows_per_req;
-          const int pos = e.pos_base[req] + i;
+          const int pos = __ldg(e.pos_base + req) + i;
           float c, sn;
-          rope_cos_sin(pos, jd % half, d, e.log2_theta, &c, &sn);
-          const float w = acc[j * kChunkLd + tp];
+          rope_cos_sin(pos, f, &c, &sn);
+          const float w = A(j, tp);
           v = jd < half ? v * c - w * sn : v * c + w * sn;
         }
         store_out(e.out[s], (size_t)m * e.ld_out[s] + n, v, e.out_bf16);
@@ -91,26 +125,27 @@ __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, in
       const int d = e.head_dim, half = d >> 1;
       const int jd = n % d, head = n / d;
       const int tp = jd < half ? t + half : t - half;
+      const double f = rope ? __ldg(e.inv_freq + jd % half) : 0.0;
       for (int j = 0; j < nrows; ++j) {
         const int m = row0 + j;
         const int req = m / e.rows_per_req, i = m % e.rows_per_req;
-        if (e.row_count && i >= e.row_count[req]) continue;
-        const int pos = e.pos_base[req] + i;
+        if (e.row_count && i >= __ldg(e.row_count + req)) continue;
+        const int pos = __ldg(e.pos_base + req) + i;
         const int slot = pos / e.page_size;
         if (pos < 0 || slot >= e.max_pages) {
           if (t == 0) flag_error(e.status, ST_BAD_PAGE);
           continue;
         }
-        const int page = e.page_table[(size_t)req * e.max_pages + slot];
+        const int page = __ldg(e.page_table + (size_t)req * e.max_pages + slot);
         if (page < 0 || page >= e.num_pages) {
           if (t == 0) flag_error(e.status, ST_BAD_PAGE);
           continue;
         }
-        float v = acc[j * kChunkLd + t];
+        float v = A(j, t);
         if (rope) {
           float c, sn;
-          rope_cos_sin(pos, jd % half, d, e.log2_theta, &c, &sn);
-          const float w = acc[j * kChunkLd + tp];
+          rope_cos_sin(pos, f, &c, &sn);
+          const float w = A(j, tp);
           v = jd < half ? v * c - w * sn : v * c + w * sn;
         }
         const size_t dst = (((size_t)page * e.n_kv + head) * e.page_size + (pos % e.page_size)) * d + jd;
@@ -119,29 +154,61 @@ __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, in
       break;
     }
     case EPI_RESID: {
+      // load every row's residual first, then add and store (independent loads in flight)
       const int n = tile * kTileN + t;
-      for (int j = 0; j < nrows; ++j) e.x[(size_t)(row0 + j) * e.ldx + n] += acc[j * kChunkLd + t];
+      float xr[kChunkRows];
+#pragma unroll
+      for (int j = 0; j < kChunkRows; ++j)
+        if (j < nrows) xr[j] = e.x[(size_t)(row0 + j) * e.ldx + n];
+      const float gn = e.xg ? __ldg(e.gamma_next + n) : 0.f;
+#pragma unroll
+      for (int j = 0; j < kChunkRows; ++j) {
+        if (j < nrows) {
+          xr[j] += A(j, t);
+          e.x[(size_t)(row0 + j) * e.ldx + n] = xr[j];
+          if (e.xg) store_out(e.xg, (size_t)(row0 + j) * e.ldx + n, xr[j] * gn, e.out_bf16);
+        }
+      }
+      if (e.sumsq) {
+        // this tile's 128 columns of each row: warp sums, then the 4 warps in order
+        float* red = scratch + kChunkRows;   // [4][32]
+        const int w = t >> 5, lane = t & 31;
+#pragma unroll
+        for (int j = 0; j < kChunkRows; ++j) {
+          const float ss = warp_sum(j < nrows ? xr[j] * xr[j] : 0.f);
+          if (lane == 0) red[w * kChunkRows + j] = ss;
+        }
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        if (t < nrows)
+          e.sumsq[(size_t)tile * e.ld_part + row0 + t] =
+              red[t] + red[kChunkRows + t] + red[2 * kChunkRows + t] + red[3 * kChunkRows + t];
+      }
       break;
     }
     case EPI_SWIGLU: {
       if (t < kTileN / 2) {
         const int f = tile * (kTileN / 2) + t;
         for (int j = 0; j < nrows; ++j) {
-          const float g = acc[j * kChunkLd + t], u = acc[j * kChunkLd + t + kTileN / 2];
+          const float g = A(j, t), u = A(j, t + kTileN / 2);
           store_out(e.out[0], (size_t)(row0 + j) * e.ld_out[0] + f, silu_f(g) * u, e.out_bf16);
         }
       }
       break;
     }
     case EPI_ARGMAX: {
-      if (t < nrows) {
-        const int vbase = tile * kTileN;
+      // warp w takes rows w, w+4, ...; each lane scans 4 of the tile's 128 vocab rows
+      const int w = t >> 5, lane = t & 31;
+      const int vbase = tile * kTileN;
+      for (int j = w; j < nrows; j += 4) {
         unsigned long long best = 0ull;
-        for (int c = 0; c < kTileN; ++c) {
-          const unsigned long long k = argmax_key(acc[t * kChunkLd + c], vbase + c);
-          best = k > best ? k : best;
+#pragma unroll
+        for (int k = 0; k < kTileN / 32; ++k) {
+          const int c = lane + 32 * k;
+          const unsigned long long key = argmax_key(A(j, c), vbase + c);
+          best = key > best ? key : best;
         }
-        atomicMax(e.keys + row0 + t, best);
+        best = warp_max_u64(best);
+        if (lane == 0) atomicMax(e.keys + row0 + j, best);
       }
       break;
     }
@@ -182,7 +249,7 @@ cudaError_t launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t 
 // Clusters of `splits` CTAs of this GEMM configuration that fit on the GPU at once.
 int gemm_tc_max_active_clusters(int m_tile, int stages, int splits);
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st);
-size_t gemm_tc_smem_bytes(int m_tile, int stages);
+size_t gemm_tc_smem_bytes(int m_tile, int stages, int splits);
 constexpr int kMaxClusterSplits = 8;
 
 }  // namespace dfl

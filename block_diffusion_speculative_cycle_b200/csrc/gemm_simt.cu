@@ -14,6 +14,7 @@ __global__ void __launch_bounds__(128) gemm_simt_kernel(const GemmSimtParams p) 
   __shared__ float xs[kChunkRows][kKT + 1];
   __shared__ float ws[kTileN][kKT + 1];
   __shared__ float chunk[kChunkRows * kChunkLd];
+  __shared__ float epi_scratch[kEpiScratch];
   const int tile = blockIdx.x;
   const int row0 = blockIdx.y * kChunkRows;
   const int t = threadIdx.x;
@@ -55,8 +56,9 @@ __global__ void __launch_bounds__(128) gemm_simt_kernel(const GemmSimtParams p) 
   }
 #pragma unroll
   for (int j = 0; j < kChunkRows; ++j) chunk[j * kChunkLd + t] = acc[j];
+  epilogue_row_scales(p.epi, row0, nrows, epi_scratch, t);
   __syncthreads();
-  epilogue_chunk(p.epi, tile, row0, nrows, chunk, t);
+  epilogue_chunk(p.epi, tile, row0, nrows, chunk, t, epi_scratch);
 }
 
 cudaError_t launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t st, bool pdl) {

@@ -9,18 +9,17 @@
 //   warp 1       TMEM owner + MMA issuer (one elected lane)
 //   warps 2..5   epilogue: TMEM -> registers -> smem chunk -> fused epilogue
 // Split-K across a thread-block cluster: the `splits` CTAs of one output tile
-// form a cluster, each reduces its own K range into TMEM, stages the fp32
-// accumulator in its shared memory, and after a cluster barrier CTA r sums rows
-// [r*m/splits, (r+1)*m/splits) over all CTAs' staging through distributed shared
-// memory, in rank order (deterministic), then runs the fused epilogue on them.
+// form a cluster and each reduces its own K range into TMEM. Rows of the tile
+// are owned in blocks of `per` by the cluster's CTAs: every CTA stages its fp32
+// partial rows in its own shared memory and bulk-copies each owner's block into
+// the owner's receive buffer (distributed shared memory, counted on the owner's
+// mbarrier); the owner waits for exactly the bytes it expects, sums the splits
+// in rank order (deterministic) and runs the fused epilogue on its rows.
 // Every mbarrier wait is bounded; on a timeout the CTA flags ST_TIMEOUT, lets
 // its copies in flight land, frees TMEM and returns.
-#include <cooperative_groups.h>
-
 #include "gemm.cuh"
 #include "sm100.cuh"
 
-namespace cg = cooperative_groups;
 
 namespace dfl {
 
@@ -32,15 +31,24 @@ constexpr int kABytes = kTileN * 64 * 2;   // 16 KB weight tile per stage
 
 __host__ __device__ inline int stage_bytes(int m_tile) { return kABytes + m_tile * 64 * 2; }
 
-size_t gemm_tc_smem_bytes(int m_tile, int stages) { return (size_t)stages * stage_bytes(m_tile) + 1024; }
+// receive buffer of the cluster reduction: splits x per x 128 fp32, per = ceil(m_tile / splits)
+__host__ __device__ inline size_t recv_bytes(int m_tile, int splits) {
+  return splits > 1 ? (size_t)splits * ((m_tile + splits - 1) / splits) * kTileN * 4 : 0;
+}
 
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmTcParams p) {
+size_t gemm_tc_smem_bytes(int m_tile, int stages, int splits) {
+  return (size_t)stages * stage_bytes(m_tile) + recv_bytes(m_tile, splits) + 1024;
+}
+
+__global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_constant__ GemmTcParams p) {
   extern __shared__ uint8_t dsmem[];
   __shared__ uint64_t full_bar[kMaxStages];
   __shared__ uint64_t empty_bar[kMaxStages];
   __shared__ uint64_t acc_bar;
+  __shared__ uint64_t recv_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int s_flag;
+  __shared__ float epi_scratch[kEpiScratch];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // blockIdx.x = ((tile * m_blocks) + mb) * splits + split; split = rank in the cluster
@@ -55,7 +63,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   const int S = p.stages;
   const int sbytes = stage_bytes(p.m_tile);
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  float* recv = reinterpret_cast<float*>(base + (size_t)S * sbytes);   // [splits][per][128]
   int* status = p.epi.status;
+  const int row0 = mb * p.m_tile;
+  const int rows_here = min(p.m_tile, p.M - row0);
+  const int per = (p.m_tile + p.splits - 1) / p.splits;
+  const int own_lo = min(rows_here, split * per), own_hi = min(rows_here, own_lo + per);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -63,8 +76,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
+    mbar_init(&recv_bar, 1);
     s_flag = 0;
     fence_mbar_init();
+    if (p.splits > 1) mbar_arrive_expect_tx(&recv_bar, (uint32_t)(p.splits * (own_hi - own_lo) * kTileN * 4));
   }
   if (warp == 0 && lane == 0) {
     if (p.paired) {
@@ -83,6 +98,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // every CTA's receive barrier is initialised before any peer may push into it
+  if (p.splits > 1) cluster_arrive_release();
 
   if (warp == 0) {
     if (lane == 0 && nkb > 0) {
@@ -156,9 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     // ------------------------------------------------------------ epilogue warps
     const int q = warp & 3;                // TMEM lane quarter this warp may access
     const int t = q * 32 + lane;           // tile row owned by this thread
-    const int row0 = mb * p.m_tile;
-    const int rows_here = min(p.m_tile, p.M - row0);
-    float* chunk = reinterpret_cast<float*>(base);
+    float* chunk = reinterpret_cast<float*>(base);   // the ring is free once the accumulator is final
     grid_dep_wait();   // epilogue reads / writes data shared with the previous kernel
     bool ok = nkb > 0 ? mbar_wait(&acc_bar, 0, status) : true;
     if (!ok) s_flag = 1;
@@ -166,68 +181,71 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     ok = (s_flag == 0) && nkb > 0;
     tc_fence_after();
     grid_dep_launch();
-    if (ok) {
-      const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-      float v[32];
-      if (p.splits == 1) {
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    float v[32];
+    if (p.splits == 1) {
+      if (ok) {
         for (int c0 = 0; c0 < rows_here; c0 += kChunkRows) {
           tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) chunk[j * kChunkLd + t] = v[j];
+          epilogue_row_scales(p.epi, row0 + c0, min(kChunkRows, rows_here - c0), epi_scratch, t);
           named_bar_sync(1, 128);
-          epilogue_chunk(p.epi, tile, row0 + c0, min(kChunkRows, rows_here - c0), chunk, t);
+          epilogue_chunk(p.epi, tile, row0 + c0, min(kChunkRows, rows_here - c0), chunk, t, epi_scratch);
           named_bar_sync(1, 128);
-        }
-      } else {
-        // stage this split's accumulator: stage[m][t], m < rows_here
-        float* stage = reinterpret_cast<float*>(base);
-        for (int c0 = 0; c0 < rows_here; c0 += kChunkRows) {
-          tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c0 + j < rows_here) stage[(c0 + j) * kTileN + t] = v[j];
         }
       }
-    } else if (p.splits > 1) {
-      // no K range (or a timed-out wait): contribute zeros
-      float* stage = reinterpret_cast<float*>(base);
-      for (int m = 0; m < rows_here; ++m) stage[m * kTileN + t] = 0.f;
+    } else {
+      // stage this split's partial rows (zeros if there was nothing to add) in the
+      // ring's memory, then bulk-copy each owner's block of rows into its receive buffer
+      cluster_wait_acquire();
+      float* stage = reinterpret_cast<float*>(base);   // [rows_here][128]
+      for (int c0 = 0; c0 < rows_here; c0 += kChunkRows) {
+        if (ok) {
+          tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < rows_here) stage[(c0 + j) * kTileN + t] = v[j];
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (t == 0) {
+        const uint32_t recv_s = smem_addr(recv), bar_s = smem_addr(&recv_bar), stage_s = smem_addr(stage);
+        for (int k = 0; k < p.splits; ++k) {
+          const int lo = min(rows_here, k * per), hi = min(rows_here, lo + per);
+          if (hi > lo)
+            bulk_copy_s2s(mapa_shared(recv_s + (uint32_t)(split * per * kTileN * 4), (uint32_t)k),
+                          stage_s + (uint32_t)(lo * kTileN * 4), (uint32_t)((hi - lo) * kTileN * 4),
+                          mapa_shared(bar_s, (uint32_t)k));
+        }
+        bulk_commit();
+      }
+      // receive: all splits' partials of the rows this CTA owns, then sum in split order
+      chunk = stage + (size_t)rows_here * kTileN;   // outgoing copies may still read the staging
+      const bool got = mbar_wait(&recv_bar, 0, status);
+      for (int c0 = own_lo; got && c0 < own_hi; c0 += kChunkRows) {
+        const int nr = min(kChunkRows, own_hi - c0);
+        for (int j = 0; j < nr; ++j) {
+          const int rl = c0 - own_lo + j;
+          float sum = 0.f;
+          for (int sp = 0; sp < p.splits; ++sp) sum += recv[(sp * per + rl) * kTileN + t];
+          chunk[j * kChunkLd + t] = sum;
+        }
+        epilogue_row_scales(p.epi, row0 + c0, nr, epi_scratch, t);
+        named_bar_sync(1, 128);
+        epilogue_chunk(p.epi, tile, row0 + c0, nr, chunk, t, epi_scratch);
+        named_bar_sync(1, 128);
+      }
+      if (t == 0) bulk_wait_read_all();   // this CTA's staging has been read by every copy
     }
     tc_fence_before();
   }
-  if (p.splits > 1) {
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();   // every split's staging is written
-    if (warp >= 2) {
-      const int t = (warp & 3) * 32 + lane;
-      const int row0 = mb * p.m_tile;
-      const int rows_here = min(p.m_tile, p.M - row0);
-      const int per = (rows_here + p.splits - 1) / p.splits;
-      const int r_lo = split * per, r_hi = min(rows_here, r_lo + per);
-      float* stage = reinterpret_cast<float*>(base);
-      float* chunk = stage + (size_t)p.m_tile * kTileN;
-      const float* rem[8];
-#pragma unroll
-      for (int s = 0; s < 8; ++s) rem[s] = s < p.splits ? cluster.map_shared_rank(stage, s) : stage;
-      for (int c0 = r_lo; c0 < r_hi; c0 += kChunkRows) {
-        const int nr = min(kChunkRows, r_hi - c0);
-        for (int j = 0; j < nr; ++j) {
-          const int off = (c0 + j) * kTileN + t;
-          float part[8];
-#pragma unroll
-          for (int s = 0; s < 8; ++s) part[s] = s < p.splits ? rem[s][off] : 0.f;
-          float sum = 0.f;
-#pragma unroll
-          for (int s = 0; s < 8; ++s) sum += part[s];
-          chunk[j * kChunkLd + t] = sum;
-        }
-        named_bar_sync(1, 128);
-        epilogue_chunk(p.epi, tile, row0 + c0, nr, chunk, t);
-        named_bar_sync(1, 128);
-      }
-    }
-    cluster.sync();   // no CTA leaves while a peer may still read its staging
-  }
+  // producer and MMA threads pass the cluster barrier they arrived at (epilogue threads already did)
+  if (p.splits > 1 && warp < 2) cluster_wait_acquire();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -236,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 }
 
 int gemm_tc_max_active_clusters(int m_tile, int stages, int splits) {
-  const size_t smem = gemm_tc_smem_bytes(m_tile, stages);
+  const size_t smem = gemm_tc_smem_bytes(m_tile, stages, splits);
   static size_t attr_bytes_q = 0;
   if (smem > attr_bytes_q) {
     if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -263,7 +281,7 @@ int gemm_tc_max_active_clusters(int m_tile, int stages, int splits) {
 }
 
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st) {
-  const size_t smem = gemm_tc_smem_bytes(p.m_tile, p.stages);
+  const size_t smem = gemm_tc_smem_bytes(p.m_tile, p.stages, p.splits);
   // the opt-in limit covers static + dynamic shared memory: raise the dynamic
   // limit only as far as this launch needs
   static size_t attr_bytes = 0;

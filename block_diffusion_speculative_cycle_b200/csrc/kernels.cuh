@@ -38,7 +38,7 @@ cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int i
 cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
                               int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
                               cudaStream_t st, bool pdl);
-// h[m] = RMSNorm(x[m]) * gain; optional fp32 copy of h into y.
+// h[m] = RMSNorm(x[m]) * gain into h (model dtype) and/or y (fp32); either may be null.
 cudaError_t launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
                            cudaStream_t st, bool pdl);
 // draft[b, i-1] = index(keys[b*B + i]) for i >= 1; every key reset to 0.

@@ -47,7 +47,7 @@ __device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
   *reinterpret_cast<uint2*>(dst) = u;
 }
 
-// h = v * rsqrt(ss/H + eps) * gain (and an fp32 copy into y if given)
+// h = v * rsqrt(ss/H + eps) * gain (h and/or an fp32 copy y, each if given)
 template <int VPT, typename HT>
 __device__ __forceinline__ void norm_store(const float4* v, float ss, int H, const float* gain, float eps, HT* h_row,
                                            float* y_row, float* red) {
@@ -61,7 +61,7 @@ __device__ __forceinline__ void norm_store(const float4* v, float ss, int H, con
     if (idx < n4) {
       const float4 g = g4[idx];
       const float4 y = make_float4(v[i].x * rstd * g.x, v[i].y * rstd * g.y, v[i].z * rstd * g.z, v[i].w * rstd * g.w);
-      store4(h_row + 4 * idx, y);
+      if (h_row) store4(h_row + 4 * idx, y);
       if (y_row) store4(y_row + 4 * idx, y);
     }
   }
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const float* x, i
   const int m = blockIdx.x;
   float4 v[VPT];
   const float ss = load_row<VPT>(x + (size_t)m * H, H, v);
-  norm_store<VPT>(v, ss, H, gain, eps, h + (size_t)m * H, y ? y + (size_t)m * H : nullptr, red);
+  norm_store<VPT>(v, ss, H, gain, eps, h ? h + (size_t)m * H : nullptr, y ? y + (size_t)m * H : nullptr, red);
 }
 
 __global__ void argmax_finalize_kernel(unsigned long long* keys, int bs, int B, int* draft) {
