@@ -155,6 +155,7 @@ struct GemmSpec {
   const void* w[kMaxSeg] = {};
   int seg_rows[kMaxSeg] = {};
   bool paired = false;
+  bool x_split = false;   // x holds hi/lo bf16 planes ([2][M][ldx]), tensor-core path only
   int tag = 0;
   EpiParams epi{};
 };
@@ -179,7 +180,8 @@ int pow2_at_least(int v) {
 dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   EpiParams& e = g.epi;
   e.status = ctx->status;
-  e.out_bf16 = ctx->bf16 ? 1 : 0;
+  e.cache_type = ctx->bf16 ? OUT_BF16 : OUT_F32;
+  if (!ctx->bf16) e.out_type = OUT_F32;
   int n_tiles = 0;
   if (g.paired) {
     n_tiles = g.seg_rows[0] / (kTileN / 2);
@@ -217,6 +219,7 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
     p.K = g.K;
     p.w_bf16 = ctx->bf16 ? 1 : 0;
     p.x_bf16 = ctx->bf16 ? 1 : 0;
+    p.x_plane = g.x_split ? (size_t)g.M * g.ldx : 0;
     p.epi = e;
     return cuda_status(launch_gemm_simt(p, n_tiles, st, ctx->use_pdl), "gemm_simt launch");
   }
@@ -226,9 +229,12 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   p.epi = e;
   p.paired = g.paired ? 1 : 0;
   p.M = g.M;
-  p.m_tile = std::min(256, (g.M + 15) / 16 * 16);
+  p.x_split = g.x_split ? 1 : 0;
+  p.x_plane_rows = g.M;
+  p.m_tile = std::min(g.x_split ? 128 : 256, (g.M + 15) / 16 * 16);
   p.m_blocks = (g.M + p.m_tile - 1) / p.m_tile;
-  p.tmem_cols = std::max(32, pow2_at_least(p.m_tile));
+  // accumulator columns: the hi plane's m_tile, then the lo plane's (read 32 at a time)
+  p.tmem_cols = std::max(32, pow2_at_least(p.x_split ? p.m_tile + (p.m_tile + 31) / 32 * 32 : p.m_tile));
   p.num_kb = g.K / 64;
   p.n_tiles = n_tiles;
   const int units = n_tiles * p.m_blocks;
@@ -238,11 +244,11 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   // third of the SM's shared memory, so three CTAs fit; otherwise use what fits.
   // The split epilogue reuses the ring for this split's rows (m_tile x 128 fp32)
   // plus one chunk; if that does not fit, use fewer splits.
-  const int sb = kTileN * 64 * 2 + p.m_tile * 128;
+  const int sb = kTileN * 64 * 2 + (1 + p.x_split) * p.m_tile * 128;
   const size_t budget = p.m_tile <= 32 ? 74 * 1024 : (p.m_tile <= 64 ? 110 * 1024 : 220 * 1024);
   const size_t chunk_bytes = (size_t)kChunkRows * kChunkLd * 4;
   for (;;) {
-    const size_t fixed = gemm_tc_smem_bytes(p.m_tile, 0, p.splits);
+    const size_t fixed = gemm_tc_smem_bytes(p.m_tile, p.x_split, 0, p.splits);
     p.stages = budget > fixed ? (int)std::min<size_t>(8, (budget - fixed) / sb) : 0;
     if (ctx->force_stages >= 2 && fixed + (size_t)ctx->force_stages * sb <= 225 * 1024) p.stages = ctx->force_stages;
     const size_t need = (p.splits > 1 ? (size_t)p.m_tile * kTileN * 4 : 0) + chunk_bytes;
@@ -259,7 +265,7 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   const int nmaps = g.paired ? 2 : g.n_seg;
   for (int s = 0; s < nmaps; ++s)
     if (!get_map(ctx, g.w[s], g.seg_rows[s], g.K, g.K, box_w, &p.wmap[s])) return DFLASH_ERR_CUDA;
-  if (!get_map(ctx, g.x, g.M, g.K, g.ldx, p.m_tile, &p.xmap)) return DFLASH_ERR_CUDA;
+  if (!get_map(ctx, g.x, (long long)(1 + p.x_split) * g.M, g.K, g.ldx, p.m_tile, &p.xmap)) return DFLASH_ERR_CUDA;
   return cuda_status(launch_gemm_tc(p, st), "gemm_tc launch");
 }
 
@@ -380,13 +386,14 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     return o;
   };
   const size_t o_x = take(R * c.hidden * 4);
-  const size_t o_h = take(R * c.hidden * es);
+  const size_t planes = ctx->bf16 ? 2 : 1;   // bf16 activations are stored as hi/lo planes
+  const size_t o_h = take(planes * R * c.hidden * es);
   const size_t o_q = take(R * q_dim(c) * es);
   const size_t o_kb = take(R * kv_dim(c) * es);
   const size_t o_vb = take(R * kv_dim(c) * es);
-  const size_t o_ao = take(R * q_dim(c) * es);
-  const size_t o_act = take(R * c.intermediate * es);
-  const size_t o_c = take(Rin * c.hidden * es);
+  const size_t o_ao = take(planes * R * q_dim(c) * es);
+  const size_t o_act = take(planes * R * c.intermediate * es);
+  const size_t o_c = take(planes * Rin * c.hidden * es);
   const size_t o_keys = take(R * 8);
   const size_t o_atto = take(ctx->att_rows * c.head_dim * 4);
   const size_t o_attm = take(ctx->att_rows * 4);
@@ -520,6 +527,8 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
   fcg.epi.kind = EPI_STORE;
   fcg.epi.out[0] = ctx->c;
   fcg.epi.ld_out[0] = c.hidden;
+  fcg.epi.out_type = OUT_BF16X2;   // c feeds the K/V GEMM as hi/lo planes
+  fcg.epi.out_plane = (size_t)M * c.hidden;
   fcg.epi.rows_per_req = max_new;
   DFL_CHECK(run_gemm(ctx, fcg, st));
 
@@ -529,6 +538,7 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
     const int nl = std::min(per_launch, c.n_layers - l0);
     GemmSpec kv;
     kv.x = ctx->c;
+    kv.x_split = ctx->bf16;
     kv.ldx = c.hidden;
     kv.M = M;
     kv.K = c.hidden;
@@ -583,7 +593,8 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
     DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, B, R, c.vocab, H,
                                             c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps,
-                                            ctx->x, ctx->h, hb, ctx->status, st, ctx->use_pdl),
+                                            ctx->x, ctx->h, hb, hb ? (size_t)R * H : 0, ctx->status, st,
+                                            ctx->use_pdl),
                           "embed_norm launch"));
   }
   const double norm_bytes = (double)R * H * (4 + es);
@@ -605,6 +616,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   for (int l = 0; l < c.n_layers; ++l) {
     GemmSpec qkv;
     qkv.x = ctx->h;
+    qkv.x_split = ctx->bf16;
     qkv.ldx = H;
     qkv.M = R;
     qkv.K = H;
@@ -617,6 +629,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     qkv.seg_rows[2] = KVD;
     qkv.tag = TAG_QKV;
     qkv.epi.kind = EPI_QKV;
+    qkv.epi.out_type = OUT_F16;   // the attention kernel runs in fp16
     qkv.epi.out[0] = ctx->q;
     qkv.epi.out[1] = ctx->kb;
     qkv.epi.out[2] = ctx->vb;
@@ -656,6 +669,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     ap.part_m = ctx->att_m;
     ap.part_l = ctx->att_l;
     ap.status = ctx->status;
+    ap.out_plane = (size_t)R * QD;
     {
       // context K/V of every request (upper bound max_ctx), block q/k/v, output
       const double kvb = (double)bs * max_ctx * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;
@@ -666,6 +680,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
 
     GemmSpec o;
     o.x = ctx->ao;
+    o.x_split = ctx->bf16;
     o.ldx = QD;
     o.M = R;
     o.K = QD;
@@ -678,6 +693,8 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     o.epi.ldx = H;
     // the MLP norm is deferred: x ⊙ gain now, the row scales in the gate/up epilogue
     o.epi.gamma_next = ctx->mlp_norm[l];
+    o.epi.out_type = OUT_BF16X2;
+    o.epi.out_plane = (size_t)R * H;
     o.epi.xg = ctx->h;
     o.epi.sumsq = ctx->sumsq[0];
     o.epi.ld_part = R;
@@ -685,6 +702,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
 
     GemmSpec gu;
     gu.x = ctx->h;
+    gu.x_split = ctx->bf16;
     gu.ldx = H;
     gu.M = R;
     gu.K = H;
@@ -695,6 +713,8 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     gu.seg_rows[0] = gu.seg_rows[1] = c.intermediate;
     gu.tag = TAG_GATEUP;
     gu.epi.kind = EPI_SWIGLU;
+    gu.epi.out_type = OUT_BF16X2;
+    gu.epi.out_plane = (size_t)R * c.intermediate;
     gu.epi.out[0] = ctx->act;
     gu.epi.ld_out[0] = c.intermediate;
     set_deferred_norm(ctx, gu.epi, ctx->sumsq[0], R);
@@ -702,6 +722,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
 
     GemmSpec dn;
     dn.x = ctx->act;
+    dn.x_split = ctx->bf16;
     dn.ldx = c.intermediate;
     dn.M = R;
     dn.K = c.intermediate;
@@ -715,6 +736,8 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     // the next layer's attention norm (or the final norm) is deferred the same way
     const bool last = l + 1 == c.n_layers;
     dn.epi.gamma_next = last ? ctx->final_norm : ctx->attn_norm[l + 1];
+    dn.epi.out_type = OUT_BF16X2;
+    dn.epi.out_plane = (size_t)R * H;
     dn.epi.xg = ctx->h;
     dn.epi.sumsq = ctx->sumsq[1];
     dn.epi.ld_part = R;
@@ -741,6 +764,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
 
   GemmSpec lm;
   lm.x = ctx->h;
+  lm.x_split = ctx->bf16;
   lm.ldx = H;
   lm.M = R;
   lm.K = H;

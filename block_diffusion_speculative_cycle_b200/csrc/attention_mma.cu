@@ -1,4 +1,4 @@
-// Tensor-core block attention (bf16 in, fp32 accumulate) for the drafter.
+// Tensor-core block attention (fp16 operands, fp32 accumulate) for the bf16 drafter.
 //
 // One CTA per (split of the key range, KV head, request); the splits of one
 // (request, KV head) form a thread-block cluster. The g*B block queries
@@ -6,14 +6,19 @@
 // split into 16-row slices, one per warp, held as mma.sync A fragments. Keys
 // stream through shared memory in tiles of 64 (a ring of 2-3 stages, cp.async 16-byte
 // copies, XOR-swizzled rows so ldmatrix is conflict-free): context keys come
-// from the request's cache pages, the B block keys from the block K/V rows.
+// from the request's cache pages (bf16), the B block keys from the block K/V
+// rows (fp16, as the QKV projection writes them). Each thread converts the
+// context chunks it copied from bf16 to fp16 in place once they land (exact for
+// |v| < 65504), so the tensor-core operands are fp16: 11 significant bits for Q,
+// the block K/V and the probabilities instead of bf16's 8.
 // Per tile: S = Q·Kᵀ (m16n8k16), online softmax in fp32 (exp2 domain, quad
 // shuffles), O += P·V with P re-packed from the S accumulators. The split's
 // state (unnormalised O, running max m, sum l) is staged per row and each block
 // of rows is bulk-copied into the receive buffer of the cluster CTA that owns
 // those rows (distributed shared memory, counted on that CTA's mbarrier); each
 // owner waits for exactly its rows, combines the splits (log-sum-exp weights,
-// split order) and writes them.
+// split order) and writes them as a pair of bf16 planes (hi, and lo = the
+// rounding residue out_plane elements further on).
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -46,17 +51,28 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t* r, const void* p) {
 }
 __device__ __forceinline__ void mma_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// Two bf16 (low half first) -> two fp16, through fp32 (a bf16 is the top half of an fp32).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  return pack_f16(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+// Write v as hi = bf16(v) at dst and lo = bf16(v - hi) at dst + plane (two elements each).
+__device__ __forceinline__ void store_split2(__nv_bfloat16* dst, size_t plane, float a, float b) {
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(hi);
+  *reinterpret_cast<__nv_bfloat162*>(dst) = hi;
+  *reinterpret_cast<__nv_bfloat162*>(dst + plane) = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+}
 
-// Element offset of (row, 8-wide chunk) in a [rows][D] bf16 tile with the
+// Element offset of (row, 8-wide chunk) in a [rows][D] 16-bit tile with the
 // 16-byte chunks of each row XOR-swizzled by row % 8.
 template <int D>
 __device__ __forceinline__ int swz(int row, int chunk) {
@@ -70,6 +86,7 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 // its own online-softmax state, merged in shared memory after the loop.
 template <int D, int NST, int KS>
 __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, __nv_bfloat16* out) {
+  const size_t plane = p.out_plane;
   constexpr int CH = D / 8;          // 16-byte chunks per row
   constexpr int REC = D + 4;         // merge record: O (D floats), m, l, two pad words (16-byte multiple)
   constexpr int NT = kKT / 8 / KS;   // score n-tiles of 8 keys per warp group
@@ -79,17 +96,17 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
   const int nr = p.g * p.B;
   const int rows_pad = ((nr + 15) / 16) * 16;
   const int slices = rows_pad / 16;
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem_raw);   // [rows_pad][D]
-  __nv_bfloat16* ring = qs + rows_pad * D;                           // NST x ([kKT][D] K, [kKT][D] V)
+  __half* qs = reinterpret_cast<__half*>(smem_raw);   // [rows_pad][D]
+  __half* ring = qs + rows_pad * D;                    // NST x ([kKT][D] K, [kKT][D] V)
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int grp = warp / slices, slice = warp % slices;
   const int gid = lane >> 2, tig = lane & 3;
   const int q_dim = p.n_q * D, kv_dim = p.n_kv * D;
-  const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q);
-  const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(p.kblk);
-  const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(p.vblk);
+  const __half* q = reinterpret_cast<const __half*>(p.q);
+  const __half* kb = reinterpret_cast<const __half*>(p.kblk);
+  const __half* vb = reinterpret_cast<const __half*>(p.vblk);
   const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(p.kc);
   const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(p.vc);
   // The context K/V were written by the injection kernels, which completed
@@ -121,9 +138,12 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
   // are one contiguous block of one page: resolve that page once.
   const bool page_tiles = (p.page_size % kKT) == 0;
   auto context_tile = [&](int kt) { return page_tiles && kt + kKT <= min(P, k1); };
+  // Chunk e of a tile (row e / CH, 16-byte chunk e % CH) is always copied by
+  // thread e % nthr, so after its own cp.async groups complete a thread can
+  // convert the context chunks it copied without a barrier.
   auto load_tile = [&](int kt, int stage) {
-    __nv_bfloat16* kd = ring + stage * 2 * kKT * D;
-    __nv_bfloat16* vd = kd + kKT * D;
+    __half* kd = ring + stage * 2 * kKT * D;
+    __half* vd = kd + kKT * D;
     if (context_tile(kt)) {
       const int slot = kt / p.page_size;
       const int page = slot < p.max_pages ? __ldg(p.page_table + (size_t)b * p.max_pages + slot) : -1;
@@ -140,8 +160,8 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     }
     for (int e = tid; e < kKT * CH; e += nthr) {
       const int r = e / CH, c = e % CH, key = kt + r;
-      const __nv_bfloat16* ksrc = kb;
-      const __nv_bfloat16* vsrc = vb;
+      const void* ksrc = kb;
+      const void* vsrc = vb;
       int bytes = 0;
       if (key < k1) {
         if (key < P) {
@@ -177,7 +197,7 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
   // Q rows r = j*B + i: query head h*g + j, block row i
   for (int e = tid; e < rows_pad * CH; e += nthr) {
     const int r = e / CH, c = e % CH;
-    const __nv_bfloat16* src = q;
+    const __half* src = q;
     int bytes = 0;
     if (r < nr) {
       const int j = r / p.B, i = r % p.B;
@@ -206,6 +226,22 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
       cp_async_wait<0>();
     else
       cp_async_wait<NST - 1>();
+    {
+      // context rows of this tile arrived as bf16: convert this thread's chunks
+      const int kt = k0 + t * kKT;
+      const int n_ctx = max(0, min(kKT, min(P, k1) - kt));
+      uint4* kd = reinterpret_cast<uint4*>(ring + (t % NST) * 2 * kKT * D);
+      uint4* vd = kd + kKT * D / 8;
+      for (int e = tid; e < n_ctx * CH; e += nthr) {
+        const int r = e / CH, c = e % CH;
+        const int o16 = swz<D>(r, c) / 8;
+        uint4 a = kd[o16], v = vd[o16];
+        a.x = bf16x2_to_f16x2(a.x); a.y = bf16x2_to_f16x2(a.y); a.z = bf16x2_to_f16x2(a.z); a.w = bf16x2_to_f16x2(a.w);
+        v.x = bf16x2_to_f16x2(v.x); v.y = bf16x2_to_f16x2(v.y); v.z = bf16x2_to_f16x2(v.z); v.w = bf16x2_to_f16x2(v.w);
+        kd[o16] = a;
+        vd[o16] = v;
+      }
+    }
     __syncthreads();
     if (active) {
       if (t == 0) {
@@ -216,8 +252,8 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
         }
       }
       const int kt = k0 + t * kKT + grp * (kKT / KS);   // this group's first key
-      const __nv_bfloat16* kt_s = ring + (t % NST) * 2 * kKT * D + grp * (kKT / KS) * D;
-      const __nv_bfloat16* vt_s = ring + (t % NST) * 2 * kKT * D + kKT * D + grp * (kKT / KS) * D;
+      const __half* kt_s = ring + (t % NST) * 2 * kKT * D + grp * (kKT / KS) * D;
+      const __half* vt_s = ring + (t % NST) * 2 * kKT * D + kKT * D + grp * (kKT / KS) * D;
       float sc[NT][4];
 #pragma unroll
       for (int n = 0; n < NT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
@@ -266,8 +302,8 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
         const float p11 = mx1 == -INFINITY ? 0.f : exp2f(sc[n][3] - m1);
         rs0 += p00 + p01;
         rs1 += p10 + p11;
-        pf[n >> 1][(n & 1) * 2 + 0] = pack_bf16(p00, p01);
-        pf[n >> 1][(n & 1) * 2 + 1] = pack_bf16(p10, p11);
+        pf[n >> 1][(n & 1) * 2 + 0] = pack_f16(p00, p01);
+        pf[n >> 1][(n & 1) * 2 + 1] = pack_f16(p10, p11);
       }
       l0 = l0 * a0 + rs0;
       l1 = l1 * a1 + rs1;
@@ -362,13 +398,13 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
         const int d = n * 8 + 2 * tig;
         if (r0 < nr) {
           const int j = r0 / p.B, i = r0 % p.B;
-          *reinterpret_cast<__nv_bfloat162*>(out + (size_t)(b * p.B + i) * q_dim + (h * p.g + j) * D + d) =
-              __floats2bfloat162_rn(o[n][0] * i0, o[n][1] * i0);
+          store_split2(out + (size_t)(b * p.B + i) * q_dim + (h * p.g + j) * D + d, plane, o[n][0] * i0,
+                       o[n][1] * i0);
         }
         if (r1 < nr) {
           const int j = r1 / p.B, i = r1 % p.B;
-          *reinterpret_cast<__nv_bfloat162*>(out + (size_t)(b * p.B + i) * q_dim + (h * p.g + j) * D + d) =
-              __floats2bfloat162_rn(o[n][2] * i1, o[n][3] * i1);
+          store_split2(out + (size_t)(b * p.B + i) * q_dim + (h * p.g + j) * D + d, plane, o[n][2] * i1,
+                       o[n][3] * i1);
         }
       }
     }
@@ -436,7 +472,12 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     const int j = r / p.B, i = r % p.B;
     __nv_bfloat16* dst = out + (size_t)(b * p.B + i) * q_dim + (h * p.g + j) * D;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) dst[lane + 32 * c] = __float2bfloat16_rn(acc[c] * invL);
+    for (int c = 0; c < D / 32; ++c) {
+      const float v = acc[c] * invL;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      dst[lane + 32 * c] = hi;
+      dst[lane + 32 * c + plane] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    }
   }
   if (tid == 0) sm100::bulk_wait_read_all();   // the staging has been read by every outgoing copy
 }

@@ -4,6 +4,8 @@
 // activation rows; its epilogue is fused (see EpiKind).
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace dfl {
@@ -36,6 +38,7 @@ struct EpiParams {
   const int* row_count;              // [bs] valid rows per request (nullptr: all)
   const int* page_table;             // [bs, max_pages]
   int max_pages, num_pages, page_size, n_kv;
+  int cache_type;                    // element type of the KV cache pools (OUT_F32 / OUT_BF16)
   float* x;                          // residual stream [M, ldx] fp32
   int ldx;
   // Deferred RMSNorm of this GEMM's input rows (the input is x ⊙ gain, not yet
@@ -52,7 +55,8 @@ struct EpiParams {
   float* sumsq;
   unsigned long long* keys;          // [M] packed argmax keys
   int* status;
-  int out_bf16;                      // 1: bf16 outputs, 0: fp32 outputs
+  int out_type;                      // OUT_F32 / OUT_BF16 / OUT_F16 / OUT_BF16X2 (see store_out)
+  size_t out_plane;                  // OUT_BF16X2: elements from the hi plane to the lo plane
 };
 
 __device__ __forceinline__ int seg_of_tile(const EpiParams& e, int tile) {
@@ -61,11 +65,28 @@ __device__ __forceinline__ int seg_of_tile(const EpiParams& e, int tile) {
   return s;
 }
 
-__device__ __forceinline__ void store_out(void* base, size_t idx, float v, int bf16) {
-  if (bf16)
-    reinterpret_cast<__nv_bfloat16*>(base)[idx] = __float2bfloat16_rn(v);
-  else
-    reinterpret_cast<float*>(base)[idx] = v;
+// Output element types. OUT_BF16X2 stores v as a pair of bf16 planes: hi = bf16(v)
+// at idx and lo = bf16(v - hi) at idx + plane, so that a GEMM reading both planes
+// as operands sees v to about 16 significant bits.
+enum OutType : int { OUT_F32 = 0, OUT_BF16 = 1, OUT_F16 = 2, OUT_BF16X2 = 3 };
+
+__device__ __forceinline__ void store_out(void* base, size_t idx, float v, int type, size_t plane = 0) {
+  switch (type) {
+    case OUT_BF16:
+      reinterpret_cast<__nv_bfloat16*>(base)[idx] = __float2bfloat16_rn(v);
+      break;
+    case OUT_F16:
+      reinterpret_cast<__half*>(base)[idx] = __float2half_rn(v);
+      break;
+    case OUT_BF16X2: {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      reinterpret_cast<__nv_bfloat16*>(base)[idx] = hi;
+      reinterpret_cast<__nv_bfloat16*>(base)[idx + plane] = __float2bfloat16_rn(v - __bfloat162float(hi));
+      break;
+    }
+    default:
+      reinterpret_cast<float*>(base)[idx] = v;
+  }
 }
 
 // Scratch of the epilogue (shared memory, per CTA): row scales, then a 4 x 32 reduction area.
@@ -114,7 +135,7 @@ __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, in
           const float w = A(j, tp);
           v = jd < half ? v * c - w * sn : v * c + w * sn;
         }
-        store_out(e.out[s], (size_t)m * e.ld_out[s] + n, v, e.out_bf16);
+        store_out(e.out[s], (size_t)m * e.ld_out[s] + n, v, e.out_type, e.out_plane);
       }
       break;
     }
@@ -149,7 +170,7 @@ __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, in
           v = jd < half ? v * c - w * sn : v * c + w * sn;
         }
         const size_t dst = (((size_t)page * e.n_kv + head) * e.page_size + (pos % e.page_size)) * d + jd;
-        store_out(e.out[s], dst, v, e.out_bf16);
+        store_out(e.out[s], dst, v, e.cache_type);
       }
       break;
     }
@@ -166,7 +187,7 @@ __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, in
         if (j < nrows) {
           xr[j] += A(j, t);
           e.x[(size_t)(row0 + j) * e.ldx + n] = xr[j];
-          if (e.xg) store_out(e.xg, (size_t)(row0 + j) * e.ldx + n, xr[j] * gn, e.out_bf16);
+          if (e.xg) store_out(e.xg, (size_t)(row0 + j) * e.ldx + n, xr[j] * gn, e.out_type, e.out_plane);
         }
       }
       if (e.sumsq) {
@@ -190,7 +211,7 @@ __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, in
         const int f = tile * (kTileN / 2) + t;
         for (int j = 0; j < nrows; ++j) {
           const float g = A(j, t), u = A(j, t + kTileN / 2);
-          store_out(e.out[0], (size_t)(row0 + j) * e.ld_out[0] + f, silu_f(g) * u, e.out_bf16);
+          store_out(e.out[0], (size_t)(row0 + j) * e.ld_out[0] + f, silu_f(g) * u, e.out_type, e.out_plane);
         }
       }
       break;
@@ -225,16 +246,19 @@ struct GemmSimtParams {
   int ldx;
   int M, K;
   int w_bf16, x_bf16;
+  size_t x_plane;           // bf16 split activations: elements to the lo plane (0: single plane)
   EpiParams epi;
 };
 
 struct alignas(64) GemmTcParams {
   CUtensorMap wmap[kMaxSeg];   // weight segment maps: box 64 (K) x 128 rows (64 rows when paired)
-  CUtensorMap xmap;            // activation map: box 64 (K) x m_tile rows
+  CUtensorMap xmap;            // activation map: box 64 (K) x m_tile rows (both planes when x_split)
   EpiParams epi;
   int paired;
   int M;                       // valid activation rows
-  int m_tile;                  // activation rows per CTA = MMA N (multiple of 16, <= 256)
+  int m_tile;                  // activation rows per CTA (multiple of 16; MMA N = (1 + x_split) * m_tile <= 256)
+  int x_split;                 // activations are hi/lo bf16 planes; the lo plane starts x_plane_rows rows on
+  int x_plane_rows;
   int m_blocks;
   int tmem_cols;
   int num_kb;                  // K / 64
@@ -249,7 +273,7 @@ cudaError_t launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t 
 // Clusters of `splits` CTAs of this GEMM configuration that fit on the GPU at once.
 int gemm_tc_max_active_clusters(int m_tile, int stages, int splits);
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st);
-size_t gemm_tc_smem_bytes(int m_tile, int stages, int splits);
+size_t gemm_tc_smem_bytes(int m_tile, int x_split, int stages, int splits);
 constexpr int kMaxClusterSplits = 8;
 
 }  // namespace dfl

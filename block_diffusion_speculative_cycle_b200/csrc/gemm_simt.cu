@@ -39,7 +39,8 @@ __global__ void __launch_bounds__(128) gemm_simt_kernel(const GemmSimtParams p) 
   for (int k0 = 0; k0 < p.K; k0 += kKT) {
     for (int e = t; e < kChunkRows * kKT; e += 128) {
       const int r = e / kKT, c = e % kKT;
-      xs[r][c] = r < nrows ? to_f32(x[(size_t)(row0 + r) * p.ldx + k0 + c]) : 0.f;
+      const size_t i = (size_t)(row0 + r) * p.ldx + k0 + c;
+      xs[r][c] = r < nrows ? to_f32(x[i]) + (p.x_plane ? to_f32(x[i + p.x_plane]) : 0.f) : 0.f;
     }
     for (int e = t; e < kTileN * kKT; e += 128) {
       const int r = e / kKT, c = e % kKT;

@@ -29,15 +29,15 @@ constexpr int kMaxStages = 8;
 constexpr int kThreads = 192;
 constexpr int kABytes = kTileN * 64 * 2;   // 16 KB weight tile per stage
 
-__host__ __device__ inline int stage_bytes(int m_tile) { return kABytes + m_tile * 64 * 2; }
+__host__ __device__ inline int stage_bytes(int m_tile, int x_split) { return kABytes + (1 + x_split) * m_tile * 64 * 2; }
 
 // receive buffer of the cluster reduction: splits x per x 128 fp32, per = ceil(m_tile / splits)
 __host__ __device__ inline size_t recv_bytes(int m_tile, int splits) {
   return splits > 1 ? (size_t)splits * ((m_tile + splits - 1) / splits) * kTileN * 4 : 0;
 }
 
-size_t gemm_tc_smem_bytes(int m_tile, int stages, int splits) {
-  return (size_t)stages * stage_bytes(m_tile) + recv_bytes(m_tile, splits) + 1024;
+size_t gemm_tc_smem_bytes(int m_tile, int x_split, int stages, int splits) {
+  return (size_t)stages * stage_bytes(m_tile, x_split) + recv_bytes(m_tile, splits) + 1024;
 }
 
 __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_constant__ GemmTcParams p) {
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
   const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
   const int nkb = kb1 - kb0;
   const int S = p.stages;
-  const int sbytes = stage_bytes(p.m_tile);
+  const int sbytes = stage_bytes(p.m_tile, p.x_split);
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   float* recv = reinterpret_cast<float*>(base + (size_t)S * sbytes);   // [splits][per][128]
   int* status = p.epi.status;
@@ -123,8 +123,12 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
         }
       }
       grid_dep_wait();
-      for (int i = 0; i < pre; ++i)
-        tma_load_2d(base + (size_t)i * sbytes + kABytes, &p.xmap, &full_bar[i], (kb0 + i) * 64, mb * p.m_tile, pol_x);
+      for (int i = 0; i < pre; ++i) {
+        uint8_t* b = base + (size_t)i * sbytes + kABytes;
+        tma_load_2d(b, &p.xmap, &full_bar[i], (kb0 + i) * 64, mb * p.m_tile, pol_x);
+        if (p.x_split)
+          tma_load_2d(b + p.m_tile * 128, &p.xmap, &full_bar[i], (kb0 + i) * 64, p.x_plane_rows + mb * p.m_tile, pol_x);
+      }
       int issued = pre;
       bool ok = true;
       for (int i = pre; i < nkb && ok; ++i) {
@@ -142,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
           tma_load_2d(a, &p.wmap[seg], &full_bar[s], kc, wrow, pol_w);
         }
         tma_load_2d(b, &p.xmap, &full_bar[s], kc, mb * p.m_tile, pol_x);
+        if (p.x_split) tma_load_2d(b + p.m_tile * 128, &p.xmap, &full_bar[s], kc, p.x_plane_rows + mb * p.m_tile, pol_x);
         ++issued;
       }
       grid_dep_launch();
@@ -150,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
     }
   } else if (warp == 1) {
     if (lane == 0 && nkb > 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, p.m_tile);
+      const uint32_t idesc = idesc_bf16_f32(128, (1 + p.x_split) * p.m_tile);
       bool ok = true;
       int i = 0;
       for (; i < nkb; ++i) {
@@ -183,10 +188,21 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
     grid_dep_launch();
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     float v[32];
+    // rows c0 .. c0+31 of this thread's tile row: the hi-plane accumulator plus,
+    // with split activations, the lo-plane one m_tile columns further on
+    auto load_rows = [&](int c0) {
+      tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, v);
+      if (p.x_split) {
+        float w[32];
+        tmem_ld_32x32b_x32(lane_base + (uint32_t)(p.m_tile + c0), w);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += w[j];
+      }
+    };
     if (p.splits == 1) {
       if (ok) {
         for (int c0 = 0; c0 < rows_here; c0 += kChunkRows) {
-          tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, v);
+          load_rows(c0);
 #pragma unroll
           for (int j = 0; j < 32; ++j) chunk[j * kChunkLd + t] = v[j];
           epilogue_row_scales(p.epi, row0 + c0, min(kChunkRows, rows_here - c0), epi_scratch, t);
@@ -202,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
       float* stage = reinterpret_cast<float*>(base);   // [rows_here][128]
       for (int c0 = 0; c0 < rows_here; c0 += kChunkRows) {
         if (ok) {
-          tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, v);
+          load_rows(c0);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -254,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
 }
 
 int gemm_tc_max_active_clusters(int m_tile, int stages, int splits) {
-  const size_t smem = gemm_tc_smem_bytes(m_tile, stages, splits);
+  const size_t smem = gemm_tc_smem_bytes(m_tile, 0, stages, splits);
   static size_t attr_bytes_q = 0;
   if (smem > attr_bytes_q) {
     if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -281,7 +297,7 @@ int gemm_tc_max_active_clusters(int m_tile, int stages, int splits) {
 }
 
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st) {
-  const size_t smem = gemm_tc_smem_bytes(p.m_tile, p.stages, p.splits);
+  const size_t smem = gemm_tc_smem_bytes(p.m_tile, p.x_split, p.stages, p.splits);
   // the opt-in limit covers static + dynamic shared memory: raise the dynamic
   // limit only as far as this launch needs
   static size_t attr_bytes = 0;

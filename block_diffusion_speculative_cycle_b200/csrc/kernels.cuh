@@ -23,10 +23,13 @@ struct AttnParams {
   float* part_m;              // [bs, n_kv, n_splits, g*B]
   float* part_l;
   int* status;
+  size_t out_plane;           // tensor-core path: elements from the output's hi plane to its lo plane
 };
 
-// Tensor-core (bf16) attention: the n_splits CTAs of one (request, KV head) form a
-// cluster and merge through distributed shared memory into out [R, n_q*d] (bf16).
+// Tensor-core attention for the bf16 drafter (q / block k / block v fp16, cache bf16):
+// the n_splits CTAs of one (request, KV head) form a cluster and merge through
+// distributed shared memory into out [R, n_q*d], written as bf16 hi/lo planes
+// out_plane elements apart.
 // kps must be a multiple of 64 and n_splits <= kMaxAttnCluster.
 constexpr int kMaxAttnCluster = 16;
 cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st, bool pdl);
@@ -35,9 +38,10 @@ cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st,
 cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st, bool pdl);
 
 // x[m] = E[token(m)] (token = anchor for block index 0, mask id otherwise), h[m] = RMSNorm(x[m]) * gain.
+// With h_plane != 0 (bf16 h), h is written as hi/lo planes h_plane elements apart.
 cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
-                              int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
-                              cudaStream_t st, bool pdl);
+                              int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
+                              int* status, cudaStream_t st, bool pdl);
 // h[m] = RMSNorm(x[m]) * gain into h (model dtype) and/or y (fp32); either may be null.
 cudaError_t launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
                            cudaStream_t st, bool pdl);

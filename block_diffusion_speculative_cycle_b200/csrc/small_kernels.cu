@@ -38,19 +38,27 @@ __device__ __forceinline__ float load_row(const float* x_row, int H, float4* v) 
   return ss;
 }
 
-__device__ __forceinline__ void store4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
-__device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
+__device__ __forceinline__ void store4(float* dst, float4 v, size_t = 0) { *reinterpret_cast<float4*>(dst) = v; }
+// bf16 rows; with plane != 0 also the lo plane bf16(v - hi) `plane` elements on
+__device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v, size_t plane = 0) {
   __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
   uint2 u;
   u.x = *reinterpret_cast<uint32_t*>(&a);
   u.y = *reinterpret_cast<uint32_t*>(&b);
   *reinterpret_cast<uint2*>(dst) = u;
+  if (plane) {
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    __nv_bfloat162 la = __floats2bfloat162_rn(v.x - fa.x, v.y - fa.y), lb = __floats2bfloat162_rn(v.z - fb.x, v.w - fb.y);
+    u.x = *reinterpret_cast<uint32_t*>(&la);
+    u.y = *reinterpret_cast<uint32_t*>(&lb);
+    *reinterpret_cast<uint2*>(dst + plane) = u;
+  }
 }
 
 // h = v * rsqrt(ss/H + eps) * gain (h and/or an fp32 copy y, each if given)
 template <int VPT, typename HT>
 __device__ __forceinline__ void norm_store(const float4* v, float ss, int H, const float* gain, float eps, HT* h_row,
-                                           float* y_row, float* red) {
+                                           float* y_row, float* red, size_t h_plane = 0) {
   ss = block_sum(ss, red);
   const float rstd = rsqrtf(ss / (float)H + eps);
   const float4* g4 = reinterpret_cast<const float4*>(gain);
@@ -61,7 +69,7 @@ __device__ __forceinline__ void norm_store(const float4* v, float ss, int H, con
     if (idx < n4) {
       const float4 g = g4[idx];
       const float4 y = make_float4(v[i].x * rstd * g.x, v[i].y * rstd * g.y, v[i].z * rstd * g.z, v[i].w * rstd * g.w);
-      if (h_row) store4(h_row + 4 * idx, y);
+      if (h_row) store4(h_row + 4 * idx, y, h_plane);
       if (y_row) store4(y_row + 4 * idx, y);
     }
   }
@@ -70,7 +78,8 @@ __device__ __forceinline__ void norm_store(const float4* v, float ss, int H, con
 template <int VPT, typename ET, typename HT>
 __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const ET* embed, const int* anchor, int mask_id,
                                                                   int B, int V, int H, const float* gain,
-                                                                  float eps, float* x, HT* h, int* status) {
+                                                                  float eps, float* x, HT* h, size_t h_plane,
+                                                                  int* status) {
   __shared__ float red[32];
   grid_dep_wait();
   grid_dep_launch();
@@ -97,7 +106,7 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const ET* embe
     if (idx < n4) store4(x + (size_t)m * H + 4 * idx, v[i]);
     ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
   }
-  norm_store<VPT>(v, ss, H, gain, eps, h + (size_t)m * H, nullptr, red);
+  norm_store<VPT>(v, ss, H, gain, eps, h + (size_t)m * H, nullptr, red, h_plane);
 }
 
 template <int VPT, typename HT>
@@ -126,33 +135,38 @@ __global__ void argmax_finalize_kernel(unsigned long long* keys, int bs, int B, 
 template <int VPT>
 static cudaError_t embed_norm_vpt(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R,
                                   int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16,
-                                  int* status, cudaStream_t st, bool pdl) {
+                                  size_t h_plane, int* status, cudaStream_t st, bool pdl) {
   const dim3 g(R), b(kNormThreads);
   if (embed_bf16 && h_bf16)
     return launch_kernel(embed_norm_kernel<VPT, __nv_bfloat16, __nv_bfloat16>, g, b, 0, st, pdl,
                          (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h,
-                         status);
+                         h_plane, status);
   if (!embed_bf16 && !h_bf16)
     return launch_kernel(embed_norm_kernel<VPT, float, float>, g, b, 0, st, pdl, (const float*)embed, anchor,
-                         mask_id, B, V, H, gain, eps, x, (float*)h, status);
+                         mask_id, B, V, H, gain, eps, x, (float*)h, (size_t)0, status);
   if (embed_bf16)
     return launch_kernel(embed_norm_kernel<VPT, __nv_bfloat16, float>, g, b, 0, st, pdl,
-                         (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (float*)h, status);
+                         (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (float*)h, (size_t)0,
+                         status);
   return launch_kernel(embed_norm_kernel<VPT, float, __nv_bfloat16>, g, b, 0, st, pdl, (const float*)embed, anchor,
-                       mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, status);
+                       mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, h_plane, status);
 }
 
 cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
-                              int H, const float* gain, float eps, float* x, void* h, int h_bf16, int* status,
-                              cudaStream_t st, bool pdl) {
+                              int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
+                              int* status, cudaStream_t st, bool pdl) {
   const int vpt = (H / 4 + kNormThreads - 1) / kNormThreads;
   if (vpt <= 1)
-    return embed_norm_vpt<1>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st, pdl);
+    return embed_norm_vpt<1>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
+                             st, pdl);
   if (vpt <= 2)
-    return embed_norm_vpt<2>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st, pdl);
+    return embed_norm_vpt<2>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
+                             st, pdl);
   if (vpt <= 4)
-    return embed_norm_vpt<4>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st, pdl);
-  return embed_norm_vpt<8>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, status, st, pdl);
+    return embed_norm_vpt<4>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
+                             st, pdl);
+  return embed_norm_vpt<8>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
+                           st, pdl);
 }
 
 template <int VPT>
