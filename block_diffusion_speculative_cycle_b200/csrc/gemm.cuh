@@ -93,148 +93,165 @@ __device__ __forceinline__ void store_out(void* base, size_t idx, float v, int t
 constexpr int kEpiScratch = kChunkRows + 4 * kChunkRows;
 
 // Row scales of the deferred RMSNorm for rows row0 .. row0+nrows-1 into
-// scratch[0..nrows): threads t < nrows each sum their row's partials in order.
-// The caller synchronises the 128 threads before epilogue_chunk reads them.
+// scratch[0..nrows): warp w takes rows w, w+4, ...; lane i sums partials i,
+// i+32, ... and a butterfly reduction (fixed order, so the result is the same
+// on every run) totals the row. All rows' loads are issued before any sum.
+// Called by the 128 epilogue threads; the caller synchronises them before the
+// epilogue reads the scales.
 __device__ __forceinline__ void epilogue_row_scales(const EpiParams& e, int row0, int nrows, float* scratch, int t) {
-  if (!e.norm_part || t >= nrows) return;
-  float ss = 0.f;
-  for (int i = 0; i < e.n_part; ++i) ss += __ldcg(e.norm_part + (size_t)i * e.ld_part + row0 + t);
-  scratch[t] = rsqrtf(ss * e.norm_inv_h + e.norm_eps);
+  if (!e.norm_part) return;
+  const int w = t >> 5, lane = t & 31;
+  float v[kChunkRows / 4];
+#pragma unroll
+  for (int r = 0; r < kChunkRows / 4; ++r) {
+    const int j = w + 4 * r;
+    float s = 0.f;
+    if (j < nrows)
+      for (int i = lane; i < e.n_part; i += 32) s += __ldcg(e.norm_part + (size_t)i * e.ld_part + row0 + j);
+    v[r] = s;
+  }
+#pragma unroll
+  for (int r = 0; r < kChunkRows / 4; ++r) {
+    const int j = w + 4 * r;
+    const float ss = warp_sum(v[r]);
+    if (j < nrows && lane == 0) scratch[j] = rsqrtf(ss * e.norm_inv_h + e.norm_eps);
+  }
 }
 
-// Apply the epilogue to one staged chunk: acc[j * kChunkLd + t] holds the
-// accumulator of activation row row0 + j (j < nrows) and tile row t (0..127),
-// scaled by scratch[j] when the input rows carry a deferred norm. Called by 128
-// threads with t = their tile row. The residual epilogue synchronises the 128
-// threads once (named barrier 2) when it produces partial sums of squares.
-__device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t,
-                                      float* scratch) {
+// Apply the epilogue of kind KIND to one staged chunk: acc[j * kChunkLd + t]
+// holds the accumulator of activation row row0 + j (j < nrows) and tile row t
+// (0..127), scaled by scratch[j] when the input rows carry a deferred norm.
+// Called by 128 threads with t = their tile row. The residual epilogue
+// synchronises the 128 threads once (named barrier 2) when it produces partial
+// sums of squares. Loops over rows are kept rolled (or lightly unrolled): the
+// epilogue runs once per CTA, so its code is fetched cold and its size, not its
+// instruction count, sets its time.
+template <int KIND>
+__device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t,
+                                        float* scratch) {
   const float* rs = e.norm_part ? scratch : nullptr;
   auto A = [&](int j, int c) -> float {
     const float v = acc[j * kChunkLd + c];
     return rs ? v * rs[j] : v;
   };
-  switch (e.kind) {
-    case EPI_STORE:
-    case EPI_QKV: {
-      const int s = seg_of_tile(e, tile);
-      const int n = (tile - e.seg_tile_begin[s]) * kTileN + t;
-      const bool rope = (e.rope_mask >> s) & 1u;
-      const int d = e.head_dim, half = d >> 1;
-      const int jd = n % d;
-      const int tp = jd < half ? t + half : t - half;
-      const double f = rope ? __ldg(e.inv_freq + jd % half) : 0.0;
-      for (int j = 0; j < nrows; ++j) {
-        const int m = row0 + j;
-        float v = A(j, t);
-        if (rope) {
-          const int req = m / e.rows_per_req, i = m % e.rows_per_req;
-          const int pos = __ldg(e.pos_base + req) + i;
-          float c, sn;
-          rope_cos_sin(pos, f, &c, &sn);
-          const float w = A(j, tp);
-          v = jd < half ? v * c - w * sn : v * c + w * sn;
-        }
-        store_out(e.out[s], (size_t)m * e.ld_out[s] + n, v, e.out_type, e.out_plane);
-      }
-      break;
-    }
-    case EPI_KV_INJECT: {
-      const int s = seg_of_tile(e, tile);
-      const int n = (tile - e.seg_tile_begin[s]) * kTileN + t;
-      const bool rope = (e.rope_mask >> s) & 1u;
-      const int d = e.head_dim, half = d >> 1;
-      const int jd = n % d, head = n / d;
-      const int tp = jd < half ? t + half : t - half;
-      const double f = rope ? __ldg(e.inv_freq + jd % half) : 0.0;
-      for (int j = 0; j < nrows; ++j) {
-        const int m = row0 + j;
+  if constexpr (KIND == EPI_STORE || KIND == EPI_QKV) {
+    const int s = seg_of_tile(e, tile);
+    const int n = (tile - e.seg_tile_begin[s]) * kTileN + t;
+    const bool rope = KIND == EPI_QKV && ((e.rope_mask >> s) & 1u);
+    const int d = e.head_dim, half = d >> 1;
+    const int jd = n % d;
+    const int tp = jd < half ? t + half : t - half;
+    const double f = rope ? __ldg(e.inv_freq + jd % half) : 0.0;
+#pragma unroll 1
+    for (int j = 0; j < nrows; ++j) {
+      const int m = row0 + j;
+      float v = A(j, t);
+      if (rope) {
         const int req = m / e.rows_per_req, i = m % e.rows_per_req;
-        if (e.row_count && i >= __ldg(e.row_count + req)) continue;
         const int pos = __ldg(e.pos_base + req) + i;
-        const int slot = pos / e.page_size;
-        if (pos < 0 || slot >= e.max_pages) {
-          if (t == 0) flag_error(e.status, ST_BAD_PAGE);
-          continue;
-        }
-        const int page = __ldg(e.page_table + (size_t)req * e.max_pages + slot);
-        if (page < 0 || page >= e.num_pages) {
-          if (t == 0) flag_error(e.status, ST_BAD_PAGE);
-          continue;
-        }
-        float v = A(j, t);
-        if (rope) {
-          float c, sn;
-          rope_cos_sin(pos, f, &c, &sn);
-          const float w = A(j, tp);
-          v = jd < half ? v * c - w * sn : v * c + w * sn;
-        }
-        const size_t dst = (((size_t)page * e.n_kv + head) * e.page_size + (pos % e.page_size)) * d + jd;
-        store_out(e.out[s], dst, v, e.cache_type);
+        float c, sn;
+        rope_cos_sin(pos, f, &c, &sn);
+        const float w = A(j, tp);
+        v = jd < half ? v * c - w * sn : v * c + w * sn;
       }
-      break;
+      store_out(e.out[s], (size_t)m * e.ld_out[s] + n, v, e.out_type, e.out_plane);
     }
-    case EPI_RESID: {
-      // load every row's residual first, then add and store (independent loads in flight)
-      const int n = tile * kTileN + t;
-      float xr[kChunkRows];
-#pragma unroll
-      for (int j = 0; j < kChunkRows; ++j)
-        if (j < nrows) xr[j] = e.x[(size_t)(row0 + j) * e.ldx + n];
-      const float gn = e.xg ? __ldg(e.gamma_next + n) : 0.f;
-#pragma unroll
-      for (int j = 0; j < kChunkRows; ++j) {
-        if (j < nrows) {
-          xr[j] += A(j, t);
-          e.x[(size_t)(row0 + j) * e.ldx + n] = xr[j];
-          if (e.xg) store_out(e.xg, (size_t)(row0 + j) * e.ldx + n, xr[j] * gn, e.out_type, e.out_plane);
-        }
+  } else if constexpr (KIND == EPI_KV_INJECT) {
+    const int s = seg_of_tile(e, tile);
+    const int n = (tile - e.seg_tile_begin[s]) * kTileN + t;
+    const bool rope = (e.rope_mask >> s) & 1u;
+    const int d = e.head_dim, half = d >> 1;
+    const int jd = n % d, head = n / d;
+    const int tp = jd < half ? t + half : t - half;
+    const double f = rope ? __ldg(e.inv_freq + jd % half) : 0.0;
+#pragma unroll 1
+    for (int j = 0; j < nrows; ++j) {
+      const int m = row0 + j;
+      const int req = m / e.rows_per_req, i = m % e.rows_per_req;
+      if (e.row_count && i >= __ldg(e.row_count + req)) continue;
+      const int pos = __ldg(e.pos_base + req) + i;
+      const int slot = pos / e.page_size;
+      if (pos < 0 || slot >= e.max_pages) {
+        if (t == 0) flag_error(e.status, ST_BAD_PAGE);
+        continue;
       }
+      const int page = __ldg(e.page_table + (size_t)req * e.max_pages + slot);
+      if (page < 0 || page >= e.num_pages) {
+        if (t == 0) flag_error(e.status, ST_BAD_PAGE);
+        continue;
+      }
+      float v = A(j, t);
+      if (rope) {
+        float c, sn;
+        rope_cos_sin(pos, f, &c, &sn);
+        const float w = A(j, tp);
+        v = jd < half ? v * c - w * sn : v * c + w * sn;
+      }
+      const size_t dst = (((size_t)page * e.n_kv + head) * e.page_size + (pos % e.page_size)) * d + jd;
+      store_out(e.out[s], dst, v, e.cache_type);
+    }
+  } else if constexpr (KIND == EPI_RESID) {
+    const int n = tile * kTileN + t;
+    const int w = t >> 5, lane = t & 31;
+    const float gn = e.xg ? __ldg(e.gamma_next + n) : 0.f;
+    float* red = scratch + kChunkRows;   // [4][kChunkRows] per-warp sums of squares
+#pragma unroll 4
+    for (int j = 0; j < nrows; ++j) {
+      float* xp = e.x + (size_t)(row0 + j) * e.ldx + n;
+      const float xv = *xp + A(j, t);
+      *xp = xv;
+      if (e.xg) store_out(e.xg, (size_t)(row0 + j) * e.ldx + n, xv * gn, e.out_type, e.out_plane);
       if (e.sumsq) {
-        // this tile's 128 columns of each row: warp sums, then the 4 warps in order
-        float* red = scratch + kChunkRows;   // [4][32]
-        const int w = t >> 5, lane = t & 31;
+        const float ss = warp_sum(xv * xv);
+        if (lane == 0) red[w * kChunkRows + j] = ss;
+      }
+    }
+    if (e.sumsq) {
+      // this tile's 128 columns of each row: the 4 warp sums in warp order
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      if (t < nrows)
+        e.sumsq[(size_t)tile * e.ld_part + row0 + t] =
+            red[t] + red[kChunkRows + t] + red[2 * kChunkRows + t] + red[3 * kChunkRows + t];
+    }
+  } else if constexpr (KIND == EPI_SWIGLU) {
+    // column c of the 64 gate / up pairs; the two thread halves take alternate rows
+    const int c = t & (kTileN / 2 - 1);
+    const int f = tile * (kTileN / 2) + c;
+#pragma unroll 2
+    for (int j = t >> 6; j < nrows; j += 2) {
+      const float g = A(j, c), u = A(j, c + kTileN / 2);
+      store_out(e.out[0], (size_t)(row0 + j) * e.ld_out[0] + f, silu_f(g) * u, e.out_type, e.out_plane);
+    }
+  } else if constexpr (KIND == EPI_ARGMAX) {
+    // warp w takes rows w, w+4, ...; each lane scans 4 of the tile's 128 vocab rows
+    const int w = t >> 5, lane = t & 31;
+    const int vbase = tile * kTileN;
+#pragma unroll 1
+    for (int j = w; j < nrows; j += 4) {
+      unsigned long long best = 0ull;
 #pragma unroll
-        for (int j = 0; j < kChunkRows; ++j) {
-          const float ss = warp_sum(j < nrows ? xr[j] * xr[j] : 0.f);
-          if (lane == 0) red[w * kChunkRows + j] = ss;
-        }
-        asm volatile("bar.sync 2, 128;" ::: "memory");
-        if (t < nrows)
-          e.sumsq[(size_t)tile * e.ld_part + row0 + t] =
-              red[t] + red[kChunkRows + t] + red[2 * kChunkRows + t] + red[3 * kChunkRows + t];
+      for (int k = 0; k < kTileN / 32; ++k) {
+        const int c = lane + 32 * k;
+        const unsigned long long key = argmax_key(A(j, c), vbase + c);
+        best = key > best ? key : best;
       }
-      break;
+      best = warp_max_u64(best);
+      if (lane == 0) atomicMax(e.keys + row0 + j, best);
     }
-    case EPI_SWIGLU: {
-      if (t < kTileN / 2) {
-        const int f = tile * (kTileN / 2) + t;
-        for (int j = 0; j < nrows; ++j) {
-          const float g = A(j, t), u = A(j, t + kTileN / 2);
-          store_out(e.out[0], (size_t)(row0 + j) * e.ld_out[0] + f, silu_f(g) * u, e.out_type, e.out_plane);
-        }
-      }
-      break;
-    }
-    case EPI_ARGMAX: {
-      // warp w takes rows w, w+4, ...; each lane scans 4 of the tile's 128 vocab rows
-      const int w = t >> 5, lane = t & 31;
-      const int vbase = tile * kTileN;
-      for (int j = w; j < nrows; j += 4) {
-        unsigned long long best = 0ull;
-#pragma unroll
-        for (int k = 0; k < kTileN / 32; ++k) {
-          const int c = lane + 32 * k;
-          const unsigned long long key = argmax_key(A(j, c), vbase + c);
-          best = key > best ? key : best;
-        }
-        best = warp_max_u64(best);
-        if (lane == 0) atomicMax(e.keys + row0 + j, best);
-      }
-      break;
-    }
-    default:
-      break;
+  }
+}
+
+// Runtime dispatch (CUDA-core GEMM).
+__device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t,
+                                      float* scratch) {
+  switch (e.kind) {
+    case EPI_STORE: epilogue_chunk_k<EPI_STORE>(e, tile, row0, nrows, acc, t, scratch); break;
+    case EPI_QKV: epilogue_chunk_k<EPI_QKV>(e, tile, row0, nrows, acc, t, scratch); break;
+    case EPI_KV_INJECT: epilogue_chunk_k<EPI_KV_INJECT>(e, tile, row0, nrows, acc, t, scratch); break;
+    case EPI_RESID: epilogue_chunk_k<EPI_RESID>(e, tile, row0, nrows, acc, t, scratch); break;
+    case EPI_SWIGLU: epilogue_chunk_k<EPI_SWIGLU>(e, tile, row0, nrows, acc, t, scratch); break;
+    case EPI_ARGMAX: epilogue_chunk_k<EPI_ARGMAX>(e, tile, row0, nrows, acc, t, scratch); break;
+    default: break;
   }
 }
 
@@ -270,8 +287,6 @@ struct alignas(64) GemmTcParams {
 };
 
 cudaError_t launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t st, bool pdl);
-// Clusters of `splits` CTAs of this GEMM configuration that fit on the GPU at once.
-int gemm_tc_max_active_clusters(int m_tile, int stages, int splits);
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st);
 size_t gemm_tc_smem_bytes(int m_tile, int x_split, int stages, int splits);
 constexpr int kMaxClusterSplits = 8;

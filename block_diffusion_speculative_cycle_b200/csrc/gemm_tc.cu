@@ -40,6 +40,8 @@ size_t gemm_tc_smem_bytes(int m_tile, int x_split, int stages, int splits) {
   return (size_t)stages * stage_bytes(m_tile, x_split) + recv_bytes(m_tile, splits) + 1024;
 }
 
+// One instantiation per epilogue kind, so a CTA fetches only its own epilogue's code.
+template <int KIND>
 __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_constant__ GemmTcParams p) {
   extern __shared__ uint8_t dsmem[];
   __shared__ uint64_t full_bar[kMaxStages];
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
           for (int j = 0; j < 32; ++j) chunk[j * kChunkLd + t] = v[j];
           epilogue_row_scales(p.epi, row0 + c0, min(kChunkRows, rows_here - c0), epi_scratch, t);
           named_bar_sync(1, 128);
-          epilogue_chunk(p.epi, tile, row0 + c0, min(kChunkRows, rows_here - c0), chunk, t, epi_scratch);
+          epilogue_chunk_k<KIND>(p.epi, tile, row0 + c0, min(kChunkRows, rows_here - c0), chunk, t, epi_scratch);
           named_bar_sync(1, 128);
         }
       }
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
         }
         epilogue_row_scales(p.epi, row0 + c0, nr, epi_scratch, t);
         named_bar_sync(1, 128);
-        epilogue_chunk(p.epi, tile, row0 + c0, nr, chunk, t, epi_scratch);
+        epilogue_chunk_k<KIND>(p.epi, tile, row0 + c0, nr, chunk, t, epi_scratch);
         named_bar_sync(1, 128);
       }
       if (t == 0) bulk_wait_read_all();   // this CTA's staging has been read by every copy
@@ -269,42 +271,25 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
   }
 }
 
-int gemm_tc_max_active_clusters(int m_tile, int stages, int splits) {
-  const size_t smem = gemm_tc_smem_bytes(m_tile, 0, stages, splits);
-  static size_t attr_bytes_q = 0;
-  if (smem > attr_bytes_q) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return 0;
-    attr_bytes_q = smem;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)splits * 64);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  return n;
-}
-
 cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st) {
   const size_t smem = gemm_tc_smem_bytes(p.m_tile, p.x_split, p.stages, p.splits);
   // the opt-in limit covers static + dynamic shared memory: raise the dynamic
   // limit only as far as this launch needs
-  static size_t attr_bytes = 0;
-  if (smem > attr_bytes) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const void* kernel = nullptr;
+  switch (p.epi.kind) {
+    case EPI_STORE: kernel = (const void*)gemm_tc_kernel<EPI_STORE>; break;
+    case EPI_QKV: kernel = (const void*)gemm_tc_kernel<EPI_QKV>; break;
+    case EPI_KV_INJECT: kernel = (const void*)gemm_tc_kernel<EPI_KV_INJECT>; break;
+    case EPI_RESID: kernel = (const void*)gemm_tc_kernel<EPI_RESID>; break;
+    case EPI_SWIGLU: kernel = (const void*)gemm_tc_kernel<EPI_SWIGLU>; break;
+    case EPI_ARGMAX: kernel = (const void*)gemm_tc_kernel<EPI_ARGMAX>; break;
+    default: return cudaErrorInvalidValue;
+  }
+  static size_t attr_bytes[EPI_ARGMAX + 1] = {};
+  if (smem > attr_bytes[p.epi.kind]) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_bytes = smem;
+    attr_bytes[p.epi.kind] = smem;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.n_tiles * p.splits * p.m_blocks));
@@ -320,7 +305,8 @@ cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st) {
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.splits > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel, p);
+  void* args[] = {const_cast<GemmTcParams*>(&p)};
+  return cudaLaunchKernelExC(&cfg, kernel, args);
 }
 
 }  // namespace dfl

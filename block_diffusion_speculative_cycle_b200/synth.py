@@ -109,6 +109,11 @@ WORKLOADS: Dict[str, Workload] = {
     "coder30b_b8_bs1": Workload("coder30b_b8_bs1", CODER_30B, block=8, batch=1, ctx_len=32768,
                                 logit_sigma=2.0, accept_mean=6.5),
 }
+# Kernel-profiling case: one Qwen3-8B-shaped layer and a 16384-row LM head, so that
+# every GEMM call site keeps its real shape (the gate/up weights alone exceed L2)
+# while the device footprint stays under 1 GB.
+WORKLOADS["qwen8b_b16_l1_v16k"] = Workload("qwen8b_b16_l1_v16k", QWEN3_8B.replace(n_layers=1, vocab=16384), block=16,
+                                           batch=1, ctx_len=2048, logit_sigma=2.0, accept_mean=6.5)
 for _bs in (1, 4, 8, 16, 32):
     WORKLOADS[f"qwen8b_b16_serve_bs{_bs}"] = Workload(
         f"qwen8b_b16_serve_bs{_bs}", QWEN3_8B, block=16, batch=_bs, ctx_range=(512, 8192),
