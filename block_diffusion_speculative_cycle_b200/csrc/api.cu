@@ -599,18 +599,26 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   }
   const double norm_bytes = (double)R * H * (4 + es);
 
-  // attention split plan
+  // attention split plan. The context of the longest request is cut into n_splits
+  // ranges of kps keys (a multiple of the kernel's key tile); the last range also
+  // takes the B block keys. Tensor-core path: the splits of one (request, KV head)
+  // form a cluster (<= 16). With few (request, KV head) pairs and <= 64 query rows
+  // the kernel runs two key groups per CTA and one wave of CTAs (one per SM);
+  // otherwise one key group and about two CTAs per SM.
   const int g = c.n_q_heads / c.n_kv_heads;
-  const int T_max = max_ctx + B;
-  // key splits: multiples of the attention kernel's key tile, about two CTAs per SM;
-  // the bf16 kernel's splits of one (request, KV head) form one cluster
+  const int pairs = bs * c.n_kv_heads;
   const int key_tile = ctx->bf16 ? 64 : 32;
-  int n_splits = std::max(1, (kAttnTargetCtas + bs * c.n_kv_heads - 1) / (bs * c.n_kv_heads));
-  if (ctx->bf16) n_splits = std::min(n_splits, kMaxAttnCluster);
-  n_splits = std::min(n_splits, (T_max + key_tile - 1) / key_tile);
-  int kps = (T_max + n_splits - 1) / n_splits;
+  int attn_ks = 1, n_splits;
+  if (ctx->bf16 && g * B <= 64 && ctx->num_sms / pairs >= 8) {
+    attn_ks = 2;
+    n_splits = std::min(kMaxAttnCluster, ctx->num_sms / pairs);
+  } else {
+    n_splits = std::max(1, (kAttnTargetCtas + pairs - 1) / pairs);
+    if (ctx->bf16) n_splits = std::min(n_splits, kMaxAttnCluster);
+  }
+  int kps = (std::max(max_ctx, 1) + n_splits - 1) / n_splits;
   kps = (kps + key_tile - 1) / key_tile * key_tile;
-  n_splits = (T_max + kps - 1) / kps;
+  n_splits = std::max(1, (max_ctx + kps - 1) / kps);
   if ((size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows) return DFLASH_ERR_UNSUPPORTED;
 
   for (int l = 0; l < c.n_layers; ++l) {
@@ -663,6 +671,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     ap.g = g;
     ap.kps = kps;
     ap.n_splits = n_splits;
+    ap.ks = attn_ks;
     ap.max_ctx = max_ctx;
     ap.scale = (float)(1.0 / std::sqrt((double)c.head_dim));
     ap.part_o = ctx->att_o;

@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
     P = P < 0 ? 0 : p.max_ctx;
   }
   const int T_all = P + p.B;
-  const int k0 = s * p.kps, k1 = min(T_all, k0 + p.kps);
+  const int k0 = s * p.kps, k1 = s == p.n_splits - 1 ? T_all : min(T_all, k0 + p.kps);
 
   for (int e = threadIdx.x; e < nr * D; e += kAttnThreads) {
     const int r = e / D, dd = e % D, j = r / p.B, i = r % p.B;

@@ -84,8 +84,12 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 // Stages of the K/V ring: 3 for up to 64 query rows, 2 for 128. KS warp groups
 // split every 64-key tile (KS = 2: group g takes keys 32g .. 32g+31), each with
 // its own online-softmax state, merged in shared memory after the loop.
+// With KS = 2 the Q fragments are re-read from shared memory for every tile
+// instead of being held in registers, so the kernel fits 128 registers and two
+// CTAs (of 256 threads) per SM: a 16-CTA cluster then needs only 8 SMs of a GPC.
 template <int D, int NST, int KS>
-__global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, __nv_bfloat16* out) {
+__global__ void __launch_bounds__(256, KS == 2 ? 2 : 0) attn_cluster_kernel(const AttnParams p, __nv_bfloat16* out) {
+  constexpr bool kQReg = KS == 1;
   const size_t plane = p.out_plane;
   constexpr int CH = D / 8;          // 16-byte chunks per row
   constexpr int REC = D + 4;         // merge record: O (D floats), m, l, two pad words (16-byte multiple)
@@ -121,7 +125,9 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     P = P < 0 ? 0 : p.max_ctx;
   }
   const int T_all = P + p.B;
-  const int k0 = s * p.kps, k1 = min(T_all, k0 + p.kps);
+  // split s takes keys [s*kps, (s+1)*kps); the last split also takes the rest
+  // (the block keys of the longest requests run up to B past n_splits*kps)
+  const int k0 = s * p.kps, k1 = s == p.n_splits - 1 ? T_all : min(T_all, k0 + p.kps);
   const int n_tiles = k1 > k0 ? (k1 - k0 + kKT - 1) / kKT : 0;
 
   const int S = p.n_splits;
@@ -141,12 +147,16 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
   // Chunk e of a tile (row e / CH, 16-byte chunk e % CH) is always copied by
   // thread e % nthr, so after its own cp.async groups complete a thread can
   // convert the context chunks it copied without a barrier.
-  auto load_tile = [&](int kt, int stage) {
+  auto tile_page = [&](int kt) {
+    const int slot = kt / p.page_size;
+    return slot < p.max_pages ? __ldg(p.page_table + (size_t)b * p.max_pages + slot) : -1;
+  };
+  // page: the tile's page when it is a context tile and the caller looked it up, else -2
+  auto load_tile = [&](int kt, int stage, int page) {
     __half* kd = ring + stage * 2 * kKT * D;
     __half* vd = kd + kKT * D;
     if (context_tile(kt)) {
-      const int slot = kt / p.page_size;
-      const int page = slot < p.max_pages ? __ldg(p.page_table + (size_t)b * p.max_pages + slot) : -1;
+      if (page == -2) page = tile_page(kt);
       const bool ok = page >= 0 && page < p.num_pages;
       if (!ok && tid == 0) flag_error(p.status, ST_BAD_PAGE);
       const size_t base = ok ? (((size_t)page * p.n_kv + h) * p.page_size + kt % p.page_size) * D : 0;
@@ -187,10 +197,14 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     }
   };
 
-  // the first NST tiles: pure-context ones now, the rest (and Q) after the wait
+  // the first NST tiles: pure-context ones now (their page ids fetched together),
+  // the rest (and Q) after the wait
+  int pg[NST];
+#pragma unroll
+  for (int i = 0; i < NST; ++i) pg[i] = i < n_tiles && context_tile(k0 + i * kKT) ? tile_page(k0 + i * kKT) : -2;
 #pragma unroll
   for (int i = 0; i < NST; ++i)
-    if (i < n_tiles && context_tile(k0 + i * kKT)) load_tile(k0 + i * kKT, i);
+    if (i < n_tiles && context_tile(k0 + i * kKT)) load_tile(k0 + i * kKT, i, pg[i]);
   cp_async_commit();
   grid_dep_wait();
   grid_dep_launch();
@@ -208,11 +222,11 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
   }
 #pragma unroll
   for (int i = 0; i < NST; ++i)
-    if (i < n_tiles && !context_tile(k0 + i * kKT)) load_tile(k0 + i * kKT, i);
+    if (i < n_tiles && !context_tile(k0 + i * kKT)) load_tile(k0 + i * kKT, i, -2);
   cp_async_commit();
 
   const bool active = slice * 16 < nr;
-  uint32_t qf[D / 16][4];
+  uint32_t qf[D / 16][4];   // used when kQReg
   const float sl2 = p.scale * 1.4426950408889634f;   // softmax in the exp2 domain
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows gid, gid+8 of this slice
   float o[D / 8][4];
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     }
     __syncthreads();
     if (active) {
-      if (t == 0) {
+      if (kQReg && t == 0) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int mat = lane >> 3, r = lane & 7;
@@ -259,14 +273,21 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
       for (int n = 0; n < NT; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
+        const int mat = lane >> 3, r = lane & 7;
+        uint32_t qt[4];
+        if constexpr (!kQReg) ldsm_x4(qt, qs + swz<D>(slice * 16 + r + 8 * (mat & 1), 2 * kk + (mat >> 1)));
 #pragma unroll
         for (int n = 0; n < NT; n += 2) {
-          const int mat = lane >> 3, r = lane & 7;
           const int kr = grp * (kKT / KS) + n * 8 + r + 8 * (mat >> 1);   // key row within the tile
           uint32_t bfr[4];
           ldsm_x4(bfr, ring + (t % NST) * 2 * kKT * D + swz<D>(kr, 2 * kk + (mat & 1)));
-          mma_16816(sc[n], qf[kk], bfr[0], bfr[1]);
-          mma_16816(sc[n + 1], qf[kk], bfr[2], bfr[3]);
+          if constexpr (kQReg) {
+            mma_16816(sc[n], qf[kk], bfr[0], bfr[1]);
+            mma_16816(sc[n + 1], qf[kk], bfr[2], bfr[3]);
+          } else {
+            mma_16816(sc[n], qt, bfr[0], bfr[1]);
+            mma_16816(sc[n + 1], qt, bfr[2], bfr[3]);
+          }
         }
       }
       (void)kt_s;
@@ -329,7 +350,7 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
       (void)vt_s;
     }
     __syncthreads();   // stage t % NST is free again
-    if (t + NST < n_tiles) load_tile(k0 + (t + NST) * kKT, t % NST);
+    if (t + NST < n_tiles) load_tile(k0 + (t + NST) * kKT, t % NST, -2);
     cp_async_commit();
   }
   cp_async_wait<0>();
@@ -346,9 +367,11 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
     }
   }
   const int r0 = slice * 16 + gid, r1 = r0 + 8;
-  float* grp_area = reinterpret_cast<float*>(smem_raw);              // [rows_pad][REC] group-1 state
-  float* stg = grp_area + (KS > 1 ? (size_t)rows_pad * REC : 0);     // [nr][REC] this split's records
-  float* rcv = stg + (size_t)nr * REC;                               // [S][per][REC] received records
+  // [rows_pad][REC]: group 1's state for the group merge, then this split's records
+  // (each group-0 thread rewrites the rows it read); [S][per][REC] received records
+  float* grp_area = reinterpret_cast<float*>(smem_raw);
+  float* stg = grp_area;
+  float* rcv = grp_area + (size_t)rows_pad * REC;
   if (KS > 1) {
     // fold the second warp group's (O, m, l) into the first group's registers
     if (active && grp == 1) {
@@ -387,6 +410,7 @@ __global__ void __launch_bounds__(256) attn_cluster_kernel(const AttnParams p, _
         mm = M;
       }
     }
+    __syncwarp();   // every lane has read its rows' m and l before they are overwritten below
   }
   const bool writer = active && grp == 0;
   if (S == 1) {
@@ -486,7 +510,7 @@ static size_t attn_cluster_smem(int d, int nr, int rows_pad, int nst, int ks, in
   const size_t loads = ((size_t)rows_pad + (size_t)nst * 2 * kKT) * d * 2;
   const size_t per = (size_t)(nr + splits - 1) / splits;
   const size_t rec = (size_t)(d + 4) * 4;
-  const size_t merge = (ks > 1 ? (size_t)rows_pad * rec : 0) + (splits > 1 ? (size_t)nr * rec + splits * per * rec : 0);
+  const size_t merge = (ks > 1 || splits > 1 ? (size_t)rows_pad * rec : 0) + (splits > 1 ? splits * per * rec : 0);
   return loads > merge ? loads : merge;
 }
 
@@ -524,9 +548,15 @@ static cudaError_t launch_cluster_t(const AttnParams& p, void* out, cudaStream_t
 
 cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {
   if (p.n_splits < 1 || p.n_splits > kMaxAttnCluster || p.kps % kKT) return cudaErrorInvalidValue;
-  // one warp per 16 query rows (one key group): two CTAs fit per SM by registers
-  // and shared memory, which keeps the clusters placeable all at once
+  // ks = 1: one warp per 16 query rows; two CTAs fit per SM by registers and
+  // shared memory, which keeps the clusters placeable all at once.
+  // ks = 2 (at most 64 query rows, grids of at most one CTA per SM): two warps
+  // per 16 rows, each taking half of every key tile, and a two-stage ring.
   const bool wide = p.g * p.B > 64;
+  if (p.ks == 2) {
+    if (wide) return cudaErrorInvalidValue;
+    return p.d == 128 ? launch_cluster_t<128, 2, 2>(p, out, st, pdl) : launch_cluster_t<64, 2, 2>(p, out, st, pdl);
+  }
   if (p.d == 128)
     return wide ? launch_cluster_t<128, 2, 1>(p, out, st, pdl) : launch_cluster_t<128, 3, 1>(p, out, st, pdl);
   return wide ? launch_cluster_t<64, 2, 1>(p, out, st, pdl) : launch_cluster_t<64, 3, 1>(p, out, st, pdl);

@@ -15,8 +15,9 @@ struct AttnParams {
   const int* page_table;      // [bs, max_pages]
   int max_pages, num_pages, page_size;
   int bs, B, n_q, n_kv, d, g;
-  int kps;                    // keys per split
+  int kps;                    // keys per split (the last split also takes the keys past n_splits*kps)
   int n_splits;
+  int ks;                     // tensor-core path: key groups per CTA (1, or 2 for <= 64 query rows)
   int max_ctx;
   float scale;                // 1/sqrt(d)
   float* part_o;              // [bs, n_kv, n_splits, g*B, d]
