@@ -93,43 +93,45 @@ __device__ __forceinline__ void store_out(void* base, size_t idx, float v, int t
 constexpr int kEpiScratch = kChunkRows + 4 * kChunkRows;
 
 // Row scales of the deferred RMSNorm for rows row0 .. row0+nrows-1 into
-// scratch[0..nrows): warp w takes rows w, w+4, ...; lane i sums partials i,
+// scale[0..nrows): warp w takes rows w, w+4, ...; lane i sums partials i,
 // i+32, ... and a butterfly reduction (fixed order, so the result is the same
-// on every run) totals the row. All rows' loads are issued before any sum.
+// on every run) totals the row. Eight rows' loads are issued before any sum.
 // Called by the 128 epilogue threads; the caller synchronises them before the
 // epilogue reads the scales.
-__device__ __forceinline__ void epilogue_row_scales(const EpiParams& e, int row0, int nrows, float* scratch, int t) {
+__device__ __forceinline__ void epilogue_row_scales(const EpiParams& e, int row0, int nrows, float* scale, int t) {
   if (!e.norm_part) return;
   const int w = t >> 5, lane = t & 31;
-  float v[kChunkRows / 4];
+  for (int base = 0; base < nrows; base += 32) {
+    float v[8];
 #pragma unroll
-  for (int r = 0; r < kChunkRows / 4; ++r) {
-    const int j = w + 4 * r;
-    float s = 0.f;
-    if (j < nrows)
-      for (int i = lane; i < e.n_part; i += 32) s += __ldcg(e.norm_part + (size_t)i * e.ld_part + row0 + j);
-    v[r] = s;
-  }
+    for (int r = 0; r < 8; ++r) {
+      const int j = base + w + 4 * r;
+      float s = 0.f;
+      if (j < nrows)
+        for (int i = lane; i < e.n_part; i += 32) s += __ldcg(e.norm_part + (size_t)i * e.ld_part + row0 + j);
+      v[r] = s;
+    }
 #pragma unroll
-  for (int r = 0; r < kChunkRows / 4; ++r) {
-    const int j = w + 4 * r;
-    const float ss = warp_sum(v[r]);
-    if (j < nrows && lane == 0) scratch[j] = rsqrtf(ss * e.norm_inv_h + e.norm_eps);
+    for (int r = 0; r < 8; ++r) {
+      const int j = base + w + 4 * r;
+      const float ss = warp_sum(v[r]);
+      if (j < nrows && lane == 0) scale[j] = rsqrtf(ss * e.norm_inv_h + e.norm_eps);
+    }
   }
 }
 
 // Apply the epilogue of kind KIND to one staged chunk: acc[j * kChunkLd + t]
 // holds the accumulator of activation row row0 + j (j < nrows) and tile row t
-// (0..127), scaled by scratch[j] when the input rows carry a deferred norm.
-// Called by 128 threads with t = their tile row. The residual epilogue
-// synchronises the 128 threads once (named barrier 2) when it produces partial
-// sums of squares. Loops over rows are kept rolled (or lightly unrolled): the
+// (0..127), scaled by rs[j] when the input rows carry a deferred norm (rs is
+// ignored otherwise). red is a [4][kChunkRows] scratch area. Called by 128
+// threads with t = their tile row. The residual epilogue synchronises the 128
+// threads once (named barrier 2) when it produces partial sums of squares. Loops over rows are kept rolled (or lightly unrolled): the
 // epilogue runs once per CTA, so its code is fetched cold and its size, not its
 // instruction count, sets its time.
 template <int KIND>
 __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t,
-                                        float* scratch) {
-  const float* rs = e.norm_part ? scratch : nullptr;
+                                        const float* rs, float* red) {
+  if (!e.norm_part) rs = nullptr;
   auto A = [&](int j, int c) -> float {
     const float v = acc[j * kChunkLd + c];
     return rs ? v * rs[j] : v;
@@ -194,7 +196,6 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
     const int n = tile * kTileN + t;
     const int w = t >> 5, lane = t & 31;
     const float gn = e.xg ? __ldg(e.gamma_next + n) : 0.f;
-    float* red = scratch + kChunkRows;   // [4][kChunkRows] per-warp sums of squares
 #pragma unroll 4
     for (int j = 0; j < nrows; ++j) {
       float* xp = e.x + (size_t)(row0 + j) * e.ldx + n;
@@ -241,16 +242,19 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
   }
 }
 
-// Runtime dispatch (CUDA-core GEMM).
+// Runtime dispatch (CUDA-core GEMM): scratch[0..kChunkRows) holds the row scales,
+// the rest the reduction area.
 __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t,
                                       float* scratch) {
+  const float* rs = scratch;
+  float* red = scratch + kChunkRows;
   switch (e.kind) {
-    case EPI_STORE: epilogue_chunk_k<EPI_STORE>(e, tile, row0, nrows, acc, t, scratch); break;
-    case EPI_QKV: epilogue_chunk_k<EPI_QKV>(e, tile, row0, nrows, acc, t, scratch); break;
-    case EPI_KV_INJECT: epilogue_chunk_k<EPI_KV_INJECT>(e, tile, row0, nrows, acc, t, scratch); break;
-    case EPI_RESID: epilogue_chunk_k<EPI_RESID>(e, tile, row0, nrows, acc, t, scratch); break;
-    case EPI_SWIGLU: epilogue_chunk_k<EPI_SWIGLU>(e, tile, row0, nrows, acc, t, scratch); break;
-    case EPI_ARGMAX: epilogue_chunk_k<EPI_ARGMAX>(e, tile, row0, nrows, acc, t, scratch); break;
+    case EPI_STORE: epilogue_chunk_k<EPI_STORE>(e, tile, row0, nrows, acc, t, rs, red); break;
+    case EPI_QKV: epilogue_chunk_k<EPI_QKV>(e, tile, row0, nrows, acc, t, rs, red); break;
+    case EPI_KV_INJECT: epilogue_chunk_k<EPI_KV_INJECT>(e, tile, row0, nrows, acc, t, rs, red); break;
+    case EPI_RESID: epilogue_chunk_k<EPI_RESID>(e, tile, row0, nrows, acc, t, rs, red); break;
+    case EPI_SWIGLU: epilogue_chunk_k<EPI_SWIGLU>(e, tile, row0, nrows, acc, t, rs, red); break;
+    case EPI_ARGMAX: epilogue_chunk_k<EPI_ARGMAX>(e, tile, row0, nrows, acc, t, rs, red); break;
     default: break;
   }
 }

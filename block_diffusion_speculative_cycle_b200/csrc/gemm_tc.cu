@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
   __shared__ uint32_t tmem_slot;
   __shared__ int s_flag;
   __shared__ float epi_scratch[kEpiScratch];
+  __shared__ float row_scale[256];   // deferred-norm scales of the tile's activation rows
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // blockIdx.x = ((tile * m_blocks) + mb) * splits + split; split = rank in the cluster
@@ -182,6 +183,8 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
     const int t = q * 32 + lane;           // tile row owned by this thread
     float* chunk = reinterpret_cast<float*>(base);   // the ring is free once the accumulator is final
     grid_dep_wait();   // epilogue reads / writes data shared with the previous kernel
+    // the row scales depend only on earlier kernels: compute them while the MMAs run
+    epilogue_row_scales(p.epi, row0, rows_here, row_scale, t);
     bool ok = nkb > 0 ? mbar_wait(&acc_bar, 0, status) : true;
     if (!ok) s_flag = 1;
     named_bar_sync(1, 128);
@@ -207,9 +210,9 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
           load_rows(c0);
 #pragma unroll
           for (int j = 0; j < 32; ++j) chunk[j * kChunkLd + t] = v[j];
-          epilogue_row_scales(p.epi, row0 + c0, min(kChunkRows, rows_here - c0), epi_scratch, t);
           named_bar_sync(1, 128);
-          epilogue_chunk_k<KIND>(p.epi, tile, row0 + c0, min(kChunkRows, rows_here - c0), chunk, t, epi_scratch);
+          epilogue_chunk_k<KIND>(p.epi, tile, row0 + c0, min(kChunkRows, rows_here - c0), chunk, t, row_scale + c0,
+                                 epi_scratch + kChunkRows);
           named_bar_sync(1, 128);
         }
       }
@@ -253,9 +256,8 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
           for (int sp = 0; sp < p.splits; ++sp) sum += recv[(sp * per + rl) * kTileN + t];
           chunk[j * kChunkLd + t] = sum;
         }
-        epilogue_row_scales(p.epi, row0 + c0, nr, epi_scratch, t);
         named_bar_sync(1, 128);
-        epilogue_chunk_k<KIND>(p.epi, tile, row0 + c0, nr, chunk, t, epi_scratch);
+        epilogue_chunk_k<KIND>(p.epi, tile, row0 + c0, nr, chunk, t, row_scale + c0, epi_scratch + kChunkRows);
         named_bar_sync(1, 128);
       }
       if (t == 0) bulk_wait_read_all();   // this CTA's staging has been read by every copy
