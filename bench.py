@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--profile-steps", type=int, default=10)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-budget-s", type=float, default=25.0)
+    ap.add_argument("--kv-cache-dtype", default="model", choices=["model", "f16"],
+                    help="element type of the drafter's KV cache pools (f16: bf16 drafters only)")
     return ap.parse_args()
 
 
@@ -148,7 +150,7 @@ def barrier(world):
 class Cycle:
     """All device state of one benchmark replica."""
 
-    def __init__(self, w, dev):
+    def __init__(self, w, dev, kv_cache_dtype="model"):
         import torch
         from block_diffusion_speculative_cycle_b200 import Drafter, dflash_verify_workspace_size, synth
         self.w, self.cfg = w, w.cfg
@@ -164,14 +166,16 @@ class Cycle:
                                                                seed=w.seed + 4)
         self.table = self.table_cpu.to(dev)
         self.max_ctx = int(self.ctx_lens.max())
-        self.drafter = Drafter(cfg, wd, max_block=B, max_batch=bs, max_inject_rows=bs * B, page_size=w.page_size)
+        cache_dt = torch.float16 if kv_cache_dtype == "f16" else cfg.torch_dtype
+        self.cache_dtype = "f16" if cache_dt == torch.float16 else cfg.dtype
+        self.drafter = Drafter(cfg, wd, max_block=B, max_batch=bs, max_inject_rows=bs * B, page_size=w.page_size,
+                               cache_dtype=cache_dt)
         # the drafter cache is filled with seeded random K/V (its values do not change the work)
         gen = torch.Generator(device=dev)
         gen.manual_seed(w.seed + 5)
         shape = (self.num_pages, cfg.n_kv_heads, w.page_size, cfg.head_dim)
-        self.kc = [torch.randn(shape, generator=gen, device=dev).mul_(2.0).to(cfg.torch_dtype)
-                   for _ in range(cfg.n_layers)]
-        self.vc = [torch.randn(shape, generator=gen, device=dev).to(cfg.torch_dtype) for _ in range(cfg.n_layers)]
+        self.kc = [torch.randn(shape, generator=gen, device=dev).mul_(2.0).to(cache_dt) for _ in range(cfg.n_layers)]
+        self.vc = [torch.randn(shape, generator=gen, device=dev).to(cache_dt) for _ in range(cfg.n_layers)]
         # step inputs
         self.feats_cpu = synth.make_features(cfg, bs * B, seed=w.seed + 1).reshape(bs, B, cfg.feat_dim)
         self.anchor_cpu = synth.make_tokens(cfg, bs, seed=w.seed + 2)
@@ -221,6 +225,27 @@ def algorithmic_cycle_bytes(c) -> float:
 
 
 # --------------------------------------------------------------------------- CPU oracle sample
+
+class HostCycle:
+    """The inputs of one cycle built on the host only (no GPU): the draft tokens
+    the logits are planted against are drawn at random instead of drafted."""
+
+    def __init__(self, w, kv_cache_dtype="model"):
+        import torch
+        from block_diffusion_speculative_cycle_b200 import synth
+        cfg, bs, B = w.cfg, w.batch, w.block
+        self.w, self.cfg, self.bs, self.B = w, cfg, bs, B
+        self.cache_dtype = "f16" if kv_cache_dtype == "f16" and cfg.dtype == "bf16" else cfg.dtype
+        self.weights_cpu = synth.make_drafter_weights(cfg, seed=w.seed)
+        self.ctx_lens = synth.make_ctx_lens(w)
+        self.feats_cpu = synth.make_features(cfg, bs * B, seed=w.seed + 1).reshape(bs, B, cfg.feat_dim)
+        self.anchor_cpu = synth.make_tokens(cfg, bs, seed=w.seed + 2)
+        self.draft = synth.make_tokens(cfg, bs * max(B - 1, 1), seed=w.seed + 3).reshape(bs, max(B - 1, 1))
+        self.logits_cpu, self.planted = synth.planted_logits(self.draft, cfg.vocab, w.logit_sigma, w.accept_mean,
+                                                             seed=w.seed + 6, dtype=torch.bfloat16)
+        self.n_new_cpu = torch.clamp(self.planted + 1, max=B).to(torch.int32)
+        self.start_cpu = (self.ctx_lens - self.n_new_cpu).clamp(min=0).to(torch.int32)
+
 
 def oracle_cycle_estimate(c, budget_s: float):
     """Time the oracle (float64 NumPy, as it stands) on a bounded sample of one
@@ -287,11 +312,8 @@ def run_reference(args, world, rank):
     w = synth.WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
 
-    class _HostOnly:
-        pass
-
     # reuse Cycle's input construction on the GPU if present (for the planted logits), else CPU-only inputs
-    c = Cycle(w, dev) if dev == "cuda" else None
+    c = Cycle(w, dev, args.kv_cache_dtype) if dev == "cuda" else HostCycle(w, args.kv_cache_dtype)
     steps = max(1, args.steps)
     budget_per_step = max(2.0, 150.0 / (steps + args.warmup))
     vals = []
@@ -319,6 +341,7 @@ def workload_config(w, c):
                         f"{cfg.n_q_heads}q/{cfg.n_kv_heads}kv x{cfg.head_dim} I{cfg.intermediate} V{cfg.vocab}, "
                         f"features {cfg.n_feat_layers}x{cfg.target_hidden}",
             "global_batch": w.batch, "block": w.block, "ctx_len": ctx, "page_size": w.page_size,
+            "kv_cache_dtype": c.cache_dtype if c is not None else cfg.dtype,
             "planted_accept_mean": w.accept_mean,
             "l2": "inputs larger than L2: every cycle streams all drafter + LM-head weights (GBs) from HBM",
             "parallelism": "replicas (one independent drafter per GPU)"}
@@ -329,7 +352,7 @@ def run_ours(args, world, rank, local):
     from block_diffusion_speculative_cycle_b200 import dflash_profile_enable, dflash_profile_read, synth
     w = synth.WORKLOADS[args.workload]
     dev = f"cuda:{local}"
-    c = Cycle(w, dev)
+    c = Cycle(w, dev, args.kv_cache_dtype)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
@@ -419,7 +442,10 @@ def run_ours(args, world, rank, local):
     # Every step copies its own inputs (features of the committed tokens, the
     # target's block logits, per-request scalars) from pinned host memory and
     # reads its results (accepted length, next token, drafts) back. Inputs are
-    # double-buffered: step k+1's copies run on a copy stream while step k computes.
+    # double-buffered: step k+1's copies run on a copy stream while step k
+    # computes. The cycle itself is the public API's inject + draft + verify,
+    # captured once per input buffer in a CUDA graph (all cycle-varying inputs are
+    # device pointers), so a step costs one graph launch on the host.
     from block_diffusion_speculative_cycle_b200 import dflash_verify
     h_feats = c.feats_cpu.pin_memory()
     h_logits = c.logits_cpu.pin_memory()
@@ -428,7 +454,21 @@ def run_ours(args, world, rank, local):
     d_feats = [torch.empty_like(c.feats) for _ in range(2)]
     d_logits = [torch.empty_like(c.logits) for _ in range(2)]
     d_small = [torch.empty_like(h_small, device=dev) for _ in range(2)]
-    comp = torch.cuda.current_stream()
+    for buf in range(2):
+        d_feats[buf].copy_(h_feats)
+        d_logits[buf].copy_(h_logits)
+        d_small[buf].copy_(h_small)
+    e2e_graphs = []
+    for buf in range(2):
+        g2 = torch.cuda.CUDAGraph()
+        sm = d_small[buf]
+        with torch.cuda.graph(g2, stream=stream):
+            c.drafter.inject(d_feats[buf], c.bs, c.B, sm[2], sm[3], c.kc, c.vc, c.table, c.num_pages)
+            c.drafter.draft(sm[0], sm[1], c.bs, c.B, c.kc, c.vc, c.table, c.num_pages, c.max_ctx, c.draft)
+            dflash_verify(d_logits[buf], c.draft, c.acc, c.nxt, c.ws)
+        e2e_graphs.append(g2)
+    torch.cuda.synchronize()
+    comp = stream
     copy = torch.cuda.Stream(device=dev)
     ev_ready = [torch.cuda.Event() for _ in range(2)]
     ev_free = [torch.cuda.Event() for _ in range(2)]
@@ -450,19 +490,17 @@ def run_ours(args, world, rank, local):
             ev_ready[buf].record(copy)
 
     stage_inputs(0)
-    for k in range(e2e_steps):
-        if k + 1 < e2e_steps:
-            stage_inputs(k + 1)
-        buf = k % 2
-        comp.wait_event(ev_ready[buf])
-        sm = d_small[buf]
-        c.drafter.inject(d_feats[buf], c.bs, c.B, sm[2], sm[3], c.kc, c.vc, c.table, c.num_pages)
-        c.drafter.draft(sm[0], sm[1], c.bs, c.B, c.kc, c.vc, c.table, c.num_pages, c.max_ctx, c.draft)
-        dflash_verify(d_logits[buf], c.draft, c.acc, c.nxt, c.ws)
-        ev_free[buf].record(comp)
-        h_out[:, 0].copy_(c.acc, non_blocking=True)
-        h_out[:, 1].copy_(c.nxt, non_blocking=True)
-        h_out[:, 2:].copy_(c.draft, non_blocking=True)
+    with torch.cuda.stream(comp):
+        for k in range(e2e_steps):
+            if k + 1 < e2e_steps:
+                stage_inputs(k + 1)
+            buf = k % 2
+            comp.wait_event(ev_ready[buf])
+            e2e_graphs[buf].replay()
+            ev_free[buf].record(comp)
+            h_out[:, 0].copy_(c.acc, non_blocking=True)
+            h_out[:, 1].copy_(c.nxt, non_blocking=True)
+            h_out[:, 2:].copy_(c.draft, non_blocking=True)
     e1.record(comp)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
@@ -493,7 +531,7 @@ def run_ours(args, world, rank, local):
                            for e in prof],
                "clocks": clk}
         print(json.dumps(out), flush=True)
-    del graph
+    del graph, e2e_graphs
 
 
 def stored_traffic(kernel: str, workload: str):

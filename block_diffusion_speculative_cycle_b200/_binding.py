@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(HERE, "libdflash.so")
 
 DFLASH_F32 = 0
 DFLASH_BF16 = 1
+DFLASH_F16 = 2
 
 _STATUS = {0: "DFLASH_OK", 1: "DFLASH_ERR_ARG", 2: "DFLASH_ERR_CUDA", 3: "DFLASH_ERR_OOM",
            4: "DFLASH_ERR_TIMEOUT", 5: "DFLASH_ERR_DEVICE", 6: "DFLASH_ERR_UNSUPPORTED"}
@@ -35,7 +36,8 @@ class dflash_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "hidden", "n_layers", "n_q_heads", "n_kv_heads", "head_dim", "intermediate", "vocab", "n_feat_layers",
         "target_hidden", "mask_token_id", "max_block", "max_batch", "max_inject_rows", "page_size")] + [
-        ("rope_theta", ctypes.c_float), ("rms_eps", ctypes.c_float), ("dtype", ctypes.c_int)]
+        ("rope_theta", ctypes.c_float), ("rms_eps", ctypes.c_float), ("dtype", ctypes.c_int),
+        ("cache_dtype", ctypes.c_int)]
 
 
 _P = ctypes.c_void_p
@@ -214,7 +216,8 @@ class Drafter:
     weights: dict with fc, embed, lm_head, final_norm and per-layer dicts (see synth)."""
 
     def __init__(self, cfg, weights: Dict, max_block: int, max_batch: int = 1, max_inject_rows: int = 64,
-                 page_size: int = 64):
+                 page_size: int = 64, cache_dtype=None):
+        import torch
         self.cfg = cfg
         self.weights = weights
         c = dflash_config()
@@ -224,6 +227,9 @@ class Drafter:
         c.max_block, c.max_batch, c.max_inject_rows, c.page_size = max_block, max_batch, max_inject_rows, page_size
         c.rope_theta, c.rms_eps = cfg.rope_theta, cfg.rms_eps
         c.dtype = DFLASH_BF16 if cfg.dtype == "bf16" else DFLASH_F32
+        # KV cache element type: the model dtype unless fp16 is asked for (bf16 drafters)
+        c.cache_dtype = DFLASH_F16 if cache_dtype == torch.float16 else c.dtype
+        self.cache_dtype = torch.float16 if cache_dtype == torch.float16 else cfg.torch_dtype
         self.config = c
         L = weights["layers"]
         self._arrays = {k: _ptr_array([lw[k] for lw in L]) for k in

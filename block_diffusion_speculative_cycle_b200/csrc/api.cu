@@ -54,10 +54,12 @@ struct dflash_ctx {
   dflash_config cfg;
   bool bf16 = false;
   bool force_simt = false;
+  bool cache_f16 = false;   // KV cache pools hold fp16 (bf16 drafter only)
   bool use_pdl = false;
   bool debug = false;
   int force_splits = 0;   // DFLASH_SPLITS: fixed K-split count (experiments)
   int force_stages = 0;   // DFLASH_STAGES: fixed ring depth (experiments)
+  int split_slots = 2;    // CTAs per SM the K-split plan fills (DFLASH_SPLIT_SLOTS, experiments)
   int num_sms = 148;
   const void* fc = nullptr;
   const void* embed = nullptr;
@@ -161,11 +163,11 @@ struct GemmSpec {
 };
 
 // K splits per output tile (= cluster size): the largest count (<= 8) that keeps
-// the grid within two CTAs per SM, so every CTA streams from the start and a
-// third slot per SM stays free for the next kernel's CTAs to start and prefetch
-// their weights (programmatic dependent launch).
+// the grid within split_slots CTAs per SM (default two), so every CTA streams
+// from the start and a third slot per SM stays free for the next kernel's CTAs
+// to start and prefetch their weights (programmatic dependent launch).
 int choose_splits(dflash_ctx* ctx, int units, int num_kb) {
-  const int slots = 2 * ctx->num_sms;
+  const int slots = ctx->split_slots * ctx->num_sms;
   for (int s = kMaxClusterSplits; s >= 2; --s)
     if (num_kb / s >= 2 && units * s <= slots) return s;
   return 1;
@@ -180,7 +182,7 @@ int pow2_at_least(int v) {
 dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   EpiParams& e = g.epi;
   e.status = ctx->status;
-  e.cache_type = ctx->bf16 ? OUT_BF16 : OUT_F32;
+  e.cache_type = ctx->cache_f16 ? OUT_F16 : (ctx->bf16 ? OUT_BF16 : OUT_F32);
   if (!ctx->bf16) e.out_type = OUT_F32;
   int n_tiles = 0;
   if (g.paired) {
@@ -311,6 +313,7 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   if (c.mask_token_id < 0 || c.mask_token_id >= c.vocab) return DFLASH_ERR_ARG;
   if (c.n_q_heads % c.n_kv_heads) return DFLASH_ERR_ARG;
   if (c.dtype != DFLASH_F32 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
+  if (c.cache_dtype == DFLASH_F16 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
   if (!w->fc || !w->embed || !w->lm_head || !w->final_norm) return DFLASH_ERR_ARG;
   if (c.n_layers > 0 && (!w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo || !w->mlp_norm || !w->wgate ||
                          !w->wup || !w->wdown))
@@ -327,6 +330,7 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   dflash_ctx* ctx = new dflash_ctx();
   ctx->cfg = c;
   ctx->bf16 = c.dtype == DFLASH_BF16;
+  ctx->cache_f16 = c.cache_dtype == DFLASH_F16;
   const char* env = std::getenv("DFLASH_FORCE_SIMT");
   ctx->force_simt = env && env[0] == '1';
   env = std::getenv("DFLASH_DEBUG");
@@ -334,6 +338,8 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
   env = std::getenv("DFLASH_SPLITS");
   ctx->force_splits = env ? std::atoi(env) : 0;
   if (ctx->force_splits > kMaxClusterSplits) ctx->force_splits = kMaxClusterSplits;
+  env = std::getenv("DFLASH_SPLIT_SLOTS");
+  if (env && std::atoi(env) >= 1 && std::atoi(env) <= 3) ctx->split_slots = std::atoi(env);
   env = std::getenv("DFLASH_STAGES");
   ctx->force_stages = env ? std::atoi(env) : 0;
   if (ctx->force_stages > 8) ctx->force_stages = 8;
@@ -679,6 +685,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     ap.part_l = ctx->att_l;
     ap.status = ctx->status;
     ap.out_plane = (size_t)R * QD;
+    ap.cache_f16 = ctx->cache_f16 ? 1 : 0;
     {
       // context K/V of every request (upper bound max_ctx), block q/k/v, output
       const double kvb = (double)bs * max_ctx * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;

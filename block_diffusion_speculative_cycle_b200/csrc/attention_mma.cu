@@ -6,11 +6,12 @@
 // split into 16-row slices, one per warp, held as mma.sync A fragments. Keys
 // stream through shared memory in tiles of 64 (a ring of 2-3 stages, cp.async 16-byte
 // copies, XOR-swizzled rows so ldmatrix is conflict-free): context keys come
-// from the request's cache pages (bf16), the B block keys from the block K/V
-// rows (fp16, as the QKV projection writes them). Each thread converts the
-// context chunks it copied from bf16 to fp16 in place once they land (exact for
-// |v| < 65504), so the tensor-core operands are fp16: 11 significant bits for Q,
-// the block K/V and the probabilities instead of bf16's 8.
+// from the request's cache pages, the B block keys from the block K/V rows
+// (fp16, as the QKV projection writes them). A bf16 cache is converted to fp16
+// in place once a tile lands, each thread converting the chunks it copied
+// (exact for |v| < 65504); an fp16 cache is used as it is. The tensor-core
+// operands are thus fp16: 11 significant bits for Q, the block K/V and the
+// probabilities instead of bf16's 8.
 // Per tile: S = Q·Kᵀ (m16n8k16), online softmax in fp32 (exp2 domain, quad
 // shuffles), O += P·V with P re-packed from the S accumulators. The split's
 // state (unnormalised O, running max m, sum l) is staged per row and each block
@@ -240,7 +241,7 @@ __global__ void __launch_bounds__(256, KS == 2 ? 2 : 0) attn_cluster_kernel(cons
       cp_async_wait<0>();
     else
       cp_async_wait<NST - 1>();
-    {
+    if (!p.cache_f16) {
       // context rows of this tile arrived as bf16: convert this thread's chunks
       const int kt = k0 + t * kKT;
       const int n_ctx = max(0, min(kKT, min(P, k1) - kt));

@@ -38,7 +38,7 @@ struct EpiParams {
   const int* row_count;              // [bs] valid rows per request (nullptr: all)
   const int* page_table;             // [bs, max_pages]
   int max_pages, num_pages, page_size, n_kv;
-  int cache_type;                    // element type of the KV cache pools (OUT_F32 / OUT_BF16)
+  int cache_type;                    // element type of the KV cache pools (OUT_F32 / OUT_BF16 / OUT_F16)
   float* x;                          // residual stream [M, ldx] fp32
   int ldx;
   // Deferred RMSNorm of this GEMM's input rows (the input is x ⊙ gain, not yet

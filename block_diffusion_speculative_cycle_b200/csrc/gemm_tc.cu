@@ -185,10 +185,9 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
     grid_dep_wait();   // epilogue reads / writes data shared with the previous kernel
     // the row scales depend only on earlier kernels: compute them while the MMAs run
     epilogue_row_scales(p.epi, row0, rows_here, row_scale, t);
-    bool ok = nkb > 0 ? mbar_wait(&acc_bar, 0, status) : true;
-    if (!ok) s_flag = 1;
-    named_bar_sync(1, 128);
-    ok = (s_flag == 0) && nkb > 0;
+    const bool got = nkb > 0 ? mbar_wait(&acc_bar, 0, status) : true;
+    // one decision for all 128 threads (the MMA lane may set s_flag at any time)
+    bool ok = !named_bar_or(1, 128, !got || s_flag != 0) && nkb > 0;
     tc_fence_after();
     grid_dep_launch();
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);

@@ -25,9 +25,10 @@ struct AttnParams {
   float* part_l;
   int* status;
   size_t out_plane;           // tensor-core path: elements from the output's hi plane to its lo plane
+  int cache_f16;              // tensor-core path: the cache pools hold fp16 (else bf16, converted on load)
 };
 
-// Tensor-core attention for the bf16 drafter (q / block k / block v fp16, cache bf16):
+// Tensor-core attention for the bf16 drafter (q / block k / block v fp16, cache bf16 or fp16):
 // the n_splits CTAs of one (request, KV head) form a cluster and merge through
 // distributed shared memory into out [R, n_q*d], written as bf16 hi/lo planes
 // out_plane elements apart.

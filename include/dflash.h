@@ -36,8 +36,9 @@
  *   - Inputs that change from cycle to cycle (anchor, context length, n_new,
  *     start position) are device pointers, so the host never needs to read
  *     the previous cycle's result.
- *   - Weights and features are bf16 or fp32 (dflash_config.dtype); RMSNorm
- *     gains are always fp32. Accumulation is fp32; the draft argmax is taken on
+ *   - Weights and features are bf16 or fp32 (dflash_config.dtype); the KV
+ *     cache is the same type or, for a bf16 drafter, fp16
+ *     (dflash_config.cache_dtype); RMSNorm gains are always fp32. Accumulation is fp32; the draft argmax is taken on
  *     fp32 logits, which are never written to memory.
  */
 #ifndef DFLASH_H
@@ -60,7 +61,7 @@ typedef enum {
   DFLASH_ERR_UNSUPPORTED = 6   /* a shape this build has no kernel for */
 } dflash_status;
 
-typedef enum { DFLASH_F32 = 0, DFLASH_BF16 = 1 } dflash_dtype;
+typedef enum { DFLASH_F32 = 0, DFLASH_BF16 = 1, DFLASH_F16 = 2 } dflash_dtype;
 
 /* Drafter shape. Notation of the pages: B = block size (anchor + B-1 masks). */
 typedef struct {
@@ -80,7 +81,13 @@ typedef struct {
   int page_size;       /* tokens per KV page (64 in the batched workloads) */
   float rope_theta;    /* rotary base theta; pair (i, i+d/2) turns by pos * theta^(-2i/d) */
   float rms_eps;       /* RMSNorm epsilon */
-  dflash_dtype dtype;  /* storage type of weights, features and the KV cache */
+  dflash_dtype dtype;  /* storage type of weights and features; DFLASH_F32 or DFLASH_BF16 */
+  /* Element type of the drafter's KV cache pools. DFLASH_F16 is accepted for a
+   * bf16 drafter: the injected K/V keep 3 more mantissa bits and the attention
+   * kernel reads them without conversion (|K|, |V| must stay below 65504). Any
+   * other value means "same as dtype" (so a zero-initialised field keeps the
+   * model dtype). DFLASH_F16 with an fp32 drafter is rejected (DFLASH_ERR_ARG). */
+  dflash_dtype cache_dtype;
 } dflash_config;
 
 /* Weights: device pointers, [out_features, in_features] row-major, in
@@ -130,7 +137,7 @@ void dflash_destroy(dflash_ctx* ctx);
  *   d_n_new     [bs] int32 (device): rows to inject per request, 0..max_new
  *   d_start_pos [bs] int32 (device): absolute position of request r's first row
  *   k_cache, v_cache: HOST arrays [n_layers] of device pointers to page pools
- *               [num_pages, n_kv, page_size, d] (dtype)
+ *               [num_pages, n_kv, page_size, d] (cache_dtype)
  *   d_page_table [bs, max_pages] int32 (device): page of token block p of request r
  * A position whose page slot is beyond max_pages, or whose page id is outside
  * [0, num_pages), is skipped and flagged (DFLASH_ERR_DEVICE). */

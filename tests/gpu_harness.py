@@ -30,19 +30,21 @@ def top2_gap(logits: np.ndarray) -> np.ndarray:
 class PagedCache:
     """Device page pools [num_pages, n_kv, page, d] per layer plus a page table."""
 
-    def __init__(self, cfg, page_table: torch.Tensor, num_pages: int, page_size: int, dev="cuda", init=None):
+    def __init__(self, cfg, page_table: torch.Tensor, num_pages: int, page_size: int, dev="cuda", init=None,
+                 dtype=None):
         self.cfg = cfg
         self.page_size = page_size
         self.num_pages = num_pages
         self.table_cpu = page_table
         self.table = page_table.to(dev)
         shape = (num_pages, cfg.n_kv_heads, page_size, cfg.head_dim)
+        dt = dtype or cfg.torch_dtype
         if init is None:
-            self.k = [torch.zeros(shape, dtype=cfg.torch_dtype, device=dev) for _ in range(cfg.n_layers)]
-            self.v = [torch.zeros(shape, dtype=cfg.torch_dtype, device=dev) for _ in range(cfg.n_layers)]
+            self.k = [torch.zeros(shape, dtype=dt, device=dev) for _ in range(cfg.n_layers)]
+            self.v = [torch.zeros(shape, dtype=dt, device=dev) for _ in range(cfg.n_layers)]
         else:
-            self.k = [lay["k"].to(dev) for lay in init]
-            self.v = [lay["v"].to(dev) for lay in init]
+            self.k = [lay["k"].to(device=dev, dtype=dt) for lay in init]
+            self.v = [lay["v"].to(device=dev, dtype=dt) for lay in init]
 
     @property
     def max_pages(self):
@@ -63,7 +65,7 @@ def gather_cpu_cache(cfg, pools_cpu, table_cpu: torch.Tensor, r: int, P: int, pa
     return O.Cache.from_arrays(cfg, ks, vs)
 
 
-def make_drafter(cfg, weights_cpu, max_block, max_batch=1, max_inject_rows=64, page_size=64):
+def make_drafter(cfg, weights_cpu, max_block, max_batch=1, max_inject_rows=64, page_size=64, cache_dtype=None):
     wd = to_dev(weights_cpu)
     return Drafter(cfg, wd, max_block=max_block, max_batch=max_batch, max_inject_rows=max_inject_rows,
-                   page_size=page_size), wd
+                   page_size=page_size, cache_dtype=cache_dtype), wd

@@ -52,3 +52,21 @@ def test_create_rejects_bad_config_without_touching_the_gpu(lib_path):
     assert lib.dflash_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)) == 1   # DFLASH_ERR_ARG
     assert lib.dflash_create(None, None, ctypes.byref(h)) == 1
     assert lib.dflash_verify(None, 0, None, 1, 4, 10, None, None, None, 0, None) == 1
+
+
+def test_drafter_config_marshalling(monkeypatch):
+    """The Drafter wrapper fills dflash_config field by field (no GPU: the C call is stubbed)."""
+    import torch
+    from block_diffusion_speculative_cycle_b200 import synth
+    seen = {}
+    monkeypatch.setattr(_binding, "dflash_create", lambda c, w: seen.setdefault("c", c) and 0)
+    cfg = synth.TINY
+    _binding.Drafter(cfg, synth.make_drafter_weights(cfg, seed=0), max_block=4, max_batch=2, max_inject_rows=8)
+    c = seen.pop("c")
+    assert (c.hidden, c.n_layers, c.max_block, c.max_batch, c.max_inject_rows) == (cfg.hidden, cfg.n_layers, 4, 2, 8)
+    assert c.dtype == _binding.DFLASH_F32 and c.cache_dtype == _binding.DFLASH_F32
+    cfg16 = cfg.replace(dtype="bf16")
+    d = _binding.Drafter(cfg16, synth.make_drafter_weights(cfg16, seed=0), max_block=4, cache_dtype=torch.float16)
+    c = seen.pop("c")
+    assert c.dtype == _binding.DFLASH_BF16 and c.cache_dtype == _binding.DFLASH_F16
+    assert d.cache_dtype == torch.float16

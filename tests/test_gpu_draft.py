@@ -19,7 +19,7 @@ SMALL_BF16 = synth.DrafterConfig(name="small-bf16", hidden=512, n_layers=2, n_q_
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 
 
-def run_case(cfg, ctx_lens, B, seed=0, chunks=1, max_new_pad=0, anchors=None, share=True):
+def run_case(cfg, ctx_lens, B, seed=0, chunks=1, max_new_pad=0, anchors=None, share=True, cache_dtype=None):
     bs = len(ctx_lens)
     ctx = torch.tensor(ctx_lens, dtype=torch.int32)
     w = synth.make_drafter_weights(cfg, seed=seed, share_embed_lm_head=share)
@@ -29,8 +29,9 @@ def run_case(cfg, ctx_lens, B, seed=0, chunks=1, max_new_pad=0, anchors=None, sh
     feats = synth.make_features(cfg, bs * max_new, seed=seed + 2).reshape(bs, max_new, cfg.feat_dim)
     if anchors is None:
         anchors = synth.make_tokens(cfg, bs, seed=seed + 3)
-    drafter, _ = make_drafter(cfg, w, max_block=B, max_batch=bs, max_inject_rows=bs * max_new, page_size=page)
-    cache = PagedCache(cfg, table, num_pages, page)
+    drafter, _ = make_drafter(cfg, w, max_block=B, max_batch=bs, max_inject_rows=bs * max_new, page_size=page,
+                              cache_dtype=cache_dtype)
+    cache = PagedCache(cfg, table, num_pages, page, dtype=cache_dtype)
 
     # GPU: inject (optionally in several chunks), then one draft pass
     dev = "cuda"
@@ -78,6 +79,13 @@ def test_tiny_fp32_ragged_batch_chunked_inject():
 @pytest.mark.parametrize("ctx_lens,B", [([200], 16), ([0, 77, 300], 10), ([1], 2), ([64, 64], 1)])
 def test_small_bf16(ctx_lens, B):
     run_case(SMALL_BF16, ctx_lens, B, seed=len(ctx_lens) + B)
+
+
+@pytest.mark.parametrize("ctx_lens,B", [([200], 16), ([0, 77, 300], 10)])
+def test_small_bf16_fp16_cache(ctx_lens, B):
+    """bf16 drafter with an fp16 KV cache: injection writes fp16 pages and the
+    attention kernel reads them without conversion."""
+    run_case(SMALL_BF16, ctx_lens, B, seed=len(ctx_lens) + B + 7, cache_dtype=torch.float16)
 
 
 def test_small_bf16_chunked_inject_and_padding_rows():

@@ -29,7 +29,7 @@ def weights_for(cfg):
     return _WEIGHTS[cfg.name]
 
 
-def run_workload(name, sample, B=None, inject_rows=16):
+def run_workload(name, sample, B=None, inject_rows=16, cache_dtype=None):
     w = synth.WORKLOADS[name]
     cfg = w.cfg
     B = B or w.block
@@ -38,10 +38,12 @@ def run_workload(name, sample, B=None, inject_rows=16):
     ctx = synth.make_ctx_lens(w)
     table, num_pages = synth.make_page_table(ctx, w.page_size, extra_tokens=max(B, inject_rows), seed=11)
     pools = synth.make_kv_cache(cfg, num_pages, w.page_size, seed=12, std=3.0)
+    if cache_dtype is not None:   # the oracle reads the same (converted) values
+        pools = [{k: t.to(cache_dtype) for k, t in lay.items()} for lay in pools]
     anchors = synth.make_tokens(cfg, bs, seed=13)
     drafter, _ = make_drafter(cfg, weights, max_block=B, max_batch=bs, max_inject_rows=bs * inject_rows,
-                              page_size=w.page_size)
-    cache = PagedCache(cfg, table, num_pages, w.page_size, init=pools)
+                              page_size=w.page_size, cache_dtype=cache_dtype)
+    cache = PagedCache(cfg, table, num_pages, w.page_size, init=pools, dtype=cache_dtype)
     dev = "cuda"
     draft = torch.zeros((bs, B - 1), dtype=torch.int32, device=dev)
     hidden = torch.zeros((cfg.n_layers + 1, bs, B, cfg.hidden), dtype=torch.float32, device=dev)
@@ -82,6 +84,10 @@ def run_workload(name, sample, B=None, inject_rows=16):
 
 def test_qwen3_8b_shaped_bs1_ctx2048_block16():
     run_workload("qwen8b_b16", sample=[0])
+
+
+def test_qwen3_8b_shaped_bs1_ctx2048_block16_fp16_cache():
+    run_workload("qwen8b_b16", sample=[0], cache_dtype=torch.float16)
 
 
 def test_llama31_8b_shaped_bs1_ctx4096_block10():
