@@ -22,6 +22,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 constexpr int kAttnTargetCtas = 296;                   // 2 CTAs per SM on 148 SMs
+constexpr int kAttnTilesPerCta = 8;                    // longest key-tile chain per attention CTA
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -608,24 +609,41 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   // attention split plan. The context of the longest request is cut into n_splits
   // ranges of kps keys (a multiple of the kernel's key tile); the last range also
   // takes the B block keys. Tensor-core path: the splits of one (request, KV head)
-  // form a cluster (<= 16). With few (request, KV head) pairs and <= 64 query rows
-  // the kernel runs two key groups per CTA and one wave of CTAs (one per SM);
-  // otherwise one key group and about two CTAs per SM.
+  // form a cluster (<= 16) and merge through distributed shared memory. With few
+  // (request, KV head) pairs and <= 64 query rows the kernel runs two key groups
+  // per CTA and one wave of CTAs (one per SM); otherwise one key group and about
+  // two CTAs per SM. Long contexts get enough splits for <= kAttnTilesPerCta key
+  // tiles per CTA; when 16 splits leave both the GPU under-filled and the CTAs
+  // long, the splits write their partials to global memory and a second kernel
+  // merges them (any split count).
   const int g = c.n_q_heads / c.n_kv_heads;
   const int pairs = bs * c.n_kv_heads;
   const int key_tile = ctx->bf16 ? 64 : 32;
+  const int ctx_tiles = std::max(1, (max_ctx + key_tile - 1) / key_tile);
   int attn_ks = 1, n_splits;
-  if (ctx->bf16 && g * B <= 64 && ctx->num_sms / pairs >= 8) {
-    attn_ks = 2;
-    n_splits = std::min(kMaxAttnCluster, ctx->num_sms / pairs);
+  bool attn_gmerge = false;
+  if (ctx->bf16) {
+    const bool small = g * B <= 64 && ctx->num_sms / pairs >= 8;
+    const int want = small ? ctx->num_sms / pairs : (kAttnTargetCtas + pairs - 1) / pairs;
+    n_splits = std::min(want, kMaxAttnCluster);
+    if (small) attn_ks = 2;
+    if ((ctx_tiles + n_splits - 1) / n_splits > kAttnTilesPerCta && pairs * kMaxAttnCluster < kAttnTargetCtas) {
+      // long context, few pairs: one wave of two-group CTAs (one per SM at 128
+      // query rows, two at <= 64), partials merged by a second kernel
+      attn_gmerge = true;
+      attn_ks = 2;
+      const int per_sm = g * B > 64 ? 1 : 2;
+      n_splits = std::min(ctx_tiles, std::max(n_splits, (per_sm * ctx->num_sms + pairs - 1) / pairs));
+    }
   } else {
     n_splits = std::max(1, (kAttnTargetCtas + pairs - 1) / pairs);
-    if (ctx->bf16) n_splits = std::min(n_splits, kMaxAttnCluster);
   }
   int kps = (std::max(max_ctx, 1) + n_splits - 1) / n_splits;
   kps = (kps + key_tile - 1) / key_tile * key_tile;
   n_splits = std::max(1, (max_ctx + kps - 1) / kps);
-  if ((size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows) return DFLASH_ERR_UNSUPPORTED;
+  // split partials in global memory (CUDA-core path, or the global merge) must fit the workspace
+  if ((!ctx->bf16 || attn_gmerge) && (size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows)
+    return DFLASH_ERR_UNSUPPORTED;
 
   for (int l = 0; l < c.n_layers; ++l) {
     GemmSpec qkv;
@@ -678,6 +696,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     ap.kps = kps;
     ap.n_splits = n_splits;
     ap.ks = attn_ks;
+    ap.global_merge = attn_gmerge ? 1 : 0;
     ap.max_ctx = max_ctx;
     ap.scale = (float)(1.0 / std::sqrt((double)c.head_dim));
     ap.part_o = ctx->att_o;

@@ -86,10 +86,12 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 // split every 64-key tile (KS = 2: group g takes keys 32g .. 32g+31), each with
 // its own online-softmax state, merged in shared memory after the loop.
 // With KS = 2 the Q fragments are re-read from shared memory for every tile
-// instead of being held in registers, so the kernel fits 128 registers and two
-// CTAs (of 256 threads) per SM: a 16-CTA cluster then needs only 8 SMs of a GPC.
+// instead of being held in registers, so the kernel fits 128 registers: two
+// CTAs of 256 threads (<= 64 query rows) per SM, so that a 16-CTA cluster needs
+// only 8 SMs of a GPC, or one CTA of 512 threads (128 query rows).
 template <int D, int NST, int KS>
-__global__ void __launch_bounds__(256, KS == 2 ? 2 : 0) attn_cluster_kernel(const AttnParams p, __nv_bfloat16* out) {
+__global__ void __launch_bounds__(KS == 2 ? 512 : 256, KS == 2 ? 1 : 0) attn_cluster_kernel(const AttnParams p,
+                                                                                            __nv_bfloat16* out) {
   constexpr bool kQReg = KS == 1;
   const size_t plane = p.out_plane;
   constexpr int CH = D / 8;          // 16-byte chunks per row
@@ -132,9 +134,11 @@ __global__ void __launch_bounds__(256, KS == 2 ? 2 : 0) attn_cluster_kernel(cons
   const int n_tiles = k1 > k0 ? (k1 - k0 + kKT - 1) / kKT : 0;
 
   const int S = p.n_splits;
+  const bool gmerge = p.global_merge != 0;   // partials to global memory, merged by a second kernel
+  if (gmerge && n_tiles == 0) return;         // a split past this request's keys: nothing to merge
   const int per = (nr + S - 1) / S;                       // merged rows owned by each split
   const int own_lo = min(nr, s * per), own_hi = min(nr, own_lo + per);
-  if (S > 1 && tid == 0) {
+  if (S > 1 && !gmerge && tid == 0) {
     sm100::mbar_init(&recv_bar, 1);
     sm100::fence_mbar_init();
     sm100::mbar_arrive_expect_tx(&recv_bar, (uint32_t)(S * (own_hi - own_lo) * REC * 4));
@@ -329,12 +333,16 @@ __global__ void __launch_bounds__(256, KS == 2 ? 2 : 0) attn_cluster_kernel(cons
       }
       l0 = l0 * a0 + rs0;
       l1 = l1 * a1 + rs1;
+      // rescale the running O only when some row's max moved (after the first
+      // tiles it rarely does); the test is warp-uniform
+      if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        o[n][0] *= a0;
-        o[n][1] *= a0;
-        o[n][2] *= a1;
-        o[n][3] *= a1;
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][0] *= a0;
+          o[n][1] *= a0;
+          o[n][2] *= a1;
+          o[n][3] *= a1;
+        }
       }
 #pragma unroll
       for (int kk = 0; kk < KK; ++kk) {
@@ -358,7 +366,7 @@ __global__ void __launch_bounds__(256, KS == 2 ? 2 : 0) attn_cluster_kernel(cons
   __syncthreads();   // every copy has landed and every warp is done with Q and the ring
   // Past this barrier Q and the ring are dead; peers may write their merge records
   // into the tail of this CTA's shared memory once every CTA of the cluster arrives.
-  if (S > 1) sm100::cluster_arrive_release();
+  if (S > 1 && !gmerge) sm100::cluster_arrive_release();
 
   if (active) {
 #pragma unroll
@@ -414,6 +422,29 @@ __global__ void __launch_bounds__(256, KS == 2 ? 2 : 0) attn_cluster_kernel(cons
     __syncwarp();   // every lane has read its rows' m and l before they are overwritten below
   }
   const bool writer = active && grp == 0;
+  if (gmerge) {
+    // this split's unnormalised O, max and sum per row (exp2 domain) for the merge kernel
+    const size_t pbase = ((size_t)(b * p.n_kv + h) * S + s) * nr;
+    if (writer) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = half ? r1 : r0;
+        if (r < nr) {
+          float* po = p.part_o + (pbase + r) * D;
+#pragma unroll
+          for (int n = 0; n < D / 8; ++n) {
+            const int d = n * 8 + 2 * tig;
+            *reinterpret_cast<float2*>(po + d) = half ? make_float2(o[n][2], o[n][3]) : make_float2(o[n][0], o[n][1]);
+          }
+          if (tig == 0) {
+            p.part_m[pbase + r] = half ? m1 : m0;
+            p.part_l[pbase + r] = half ? l1 : l0;
+          }
+        }
+      }
+    }
+    return;
+  }
   if (S == 1) {
     // the whole key range is here: normalise and write
     if (writer) {
@@ -507,12 +538,70 @@ __global__ void __launch_bounds__(256, KS == 2 ? 2 : 0) attn_cluster_kernel(cons
   if (tid == 0) sm100::bulk_wait_read_all();   // the staging has been read by every outgoing copy
 }
 
-static size_t attn_cluster_smem(int d, int nr, int rows_pad, int nst, int ks, int splits) {
+static size_t attn_cluster_smem(int d, int nr, int rows_pad, int nst, int ks, int splits, bool gmerge) {
   const size_t loads = ((size_t)rows_pad + (size_t)nst * 2 * kKT) * d * 2;
   const size_t per = (size_t)(nr + splits - 1) / splits;
   const size_t rec = (size_t)(d + 4) * 4;
-  const size_t merge = (ks > 1 || splits > 1 ? (size_t)rows_pad * rec : 0) + (splits > 1 ? splits * per * rec : 0);
+  const bool cl = splits > 1 && !gmerge;
+  const size_t merge = (ks > 1 || cl ? (size_t)rows_pad * rec : 0) + (cl ? splits * per * rec : 0);
   return loads > merge ? loads : merge;
+}
+
+// Global merge (many splits): one warp per (block row, query head) combines the
+// splits that hold keys (log-sum-exp weights in the exp2 domain, split order)
+// and writes the row as bf16 hi/lo planes.
+template <int D>
+__global__ void __launch_bounds__(256) attn_gmerge_kernel(const AttnParams p, __nv_bfloat16* out) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int R = p.bs * p.B;
+  if (gw >= R * p.n_q) return;
+  const int m_row = gw / p.n_q, j = gw % p.n_q;
+  const int b = m_row / p.B, i = m_row % p.B;
+  const int h = j / p.g, jj = j % p.g;
+  const int nr = p.g * p.B, r = jj * p.B + i;
+  int P = p.ctx_len[b];
+  P = P < 0 ? 0 : (P > p.max_ctx ? p.max_ctx : P);
+  const int used = min(p.n_splits, (P + p.B + p.kps - 1) / p.kps);
+  const size_t base = (size_t)(b * p.n_kv + h) * p.n_splits * nr + r;
+  float M = -INFINITY;
+  for (int s = lane; s < used; s += 32) M = fmaxf(M, __ldcg(p.part_m + base + (size_t)s * nr));
+  M = warp_max(M);
+  float L = 0.f;
+  for (int s = lane; s < used; s += 32) {
+    const size_t idx = base + (size_t)s * nr;
+    const float ms = __ldcg(p.part_m + idx);
+    L += ms == -INFINITY ? 0.f : __ldcg(p.part_l + idx) * exp2f(ms - M);
+  }
+  L = warp_sum(L);
+  const float invL = 1.f / L;
+  float acc[D / 32];
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
+  for (int s0 = 0; s0 < used; s0 += 32) {
+    const int sl = s0 + lane;
+    float wl = 0.f;
+    if (sl < used) {
+      const float ms = __ldcg(p.part_m + base + (size_t)sl * nr);
+      wl = ms == -INFINITY ? 0.f : exp2f(ms - M) * invL;
+    }
+    const int n = min(32, used - s0);
+#pragma unroll 4
+    for (int k = 0; k < n; ++k) {
+      const float w = __shfl_sync(0xffffffffu, wl, k);
+      const float* o = p.part_o + (base + (size_t)(s0 + k) * nr) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(w, __ldcg(o + lane + 32 * c), acc[c]);
+    }
+  }
+  __nv_bfloat16* dst = out + (size_t)m_row * p.n_q * D + j * D;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(acc[c]);
+    dst[lane + 32 * c] = hi;
+    dst[lane + 32 * c + p.out_plane] = __float2bfloat16_rn(acc[c] - __bfloat162float(hi));
+  }
 }
 
 template <int D, int NST, int KS>
@@ -520,7 +609,8 @@ static cudaError_t launch_cluster_t(const AttnParams& p, void* out, cudaStream_t
   const int nr = p.g * p.B;
   const int rows_pad = ((nr + 15) / 16) * 16;
   const int threads = 32 * KS * (rows_pad / 16);
-  const size_t smem = attn_cluster_smem(D, nr, rows_pad, NST, KS, p.n_splits);
+  const bool gmerge = p.global_merge != 0;
+  const size_t smem = attn_cluster_smem(D, nr, rows_pad, NST, KS, p.n_splits, gmerge);
   static size_t set = 0;
   if (smem > set) {
     cudaError_t e = cudaFuncSetAttribute(attn_cluster_kernel<D, NST, KS>,
@@ -543,21 +633,22 @@ static cudaError_t launch_cluster_t(const AttnParams& p, void* out, cudaStream_t
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = p.n_splits > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, attn_cluster_kernel<D, NST, KS>, p, (__nv_bfloat16*)out);
+  cfg.numAttrs = p.n_splits > 1 && !gmerge ? 2 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_cluster_kernel<D, NST, KS>, p, (__nv_bfloat16*)out);
+  if (e != cudaSuccess || !gmerge) return e;
+  const int warps = p.bs * p.B * p.n_q;
+  return launch_kernel(attn_gmerge_kernel<D>, dim3((warps + 7) / 8), dim3(256), 0, st, pdl, p, (__nv_bfloat16*)out);
 }
 
 cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {
-  if (p.n_splits < 1 || p.n_splits > kMaxAttnCluster || p.kps % kKT) return cudaErrorInvalidValue;
+  if (p.n_splits < 1 || (!p.global_merge && p.n_splits > kMaxAttnCluster) || p.kps % kKT) return cudaErrorInvalidValue;
   // ks = 1: one warp per 16 query rows; two CTAs fit per SM by registers and
   // shared memory, which keeps the clusters placeable all at once.
-  // ks = 2 (at most 64 query rows, grids of at most one CTA per SM): two warps
-  // per 16 rows, each taking half of every key tile, and a two-stage ring.
+  // ks = 2 (small grids): two warps per 16 rows, each taking half of every key
+  // tile, and a two-stage ring.
   const bool wide = p.g * p.B > 64;
-  if (p.ks == 2) {
-    if (wide) return cudaErrorInvalidValue;
+  if (p.ks == 2)
     return p.d == 128 ? launch_cluster_t<128, 2, 2>(p, out, st, pdl) : launch_cluster_t<64, 2, 2>(p, out, st, pdl);
-  }
   if (p.d == 128)
     return wide ? launch_cluster_t<128, 2, 1>(p, out, st, pdl) : launch_cluster_t<128, 3, 1>(p, out, st, pdl);
   return wide ? launch_cluster_t<64, 2, 1>(p, out, st, pdl) : launch_cluster_t<64, 3, 1>(p, out, st, pdl);

@@ -26,6 +26,7 @@ struct AttnParams {
   int* status;
   size_t out_plane;           // tensor-core path: elements from the output's hi plane to its lo plane
   int cache_f16;              // tensor-core path: the cache pools hold fp16 (else bf16, converted on load)
+  int global_merge;           // tensor-core path: splits write part_o/m/l (exp2 domain) and a second kernel merges
 };
 
 // Tensor-core attention for the bf16 drafter (q / block k / block v fp16, cache bf16 or fp16):
