@@ -626,12 +626,11 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     const bool small = g * B <= 64 && ctx->num_sms / pairs >= 8;
     const int want = small ? ctx->num_sms / pairs : (kAttnTargetCtas + pairs - 1) / pairs;
     n_splits = std::min(want, kMaxAttnCluster);
-    if (small) attn_ks = 2;
+    attn_ks = 2;   // two key groups per CTA (two CTAs per SM at <= 64 query rows, one at 128)
     if ((ctx_tiles + n_splits - 1) / n_splits > kAttnTilesPerCta && pairs * kMaxAttnCluster < kAttnTargetCtas) {
       // long context, few pairs: one wave of two-group CTAs (one per SM at 128
       // query rows, two at <= 64), partials merged by a second kernel
       attn_gmerge = true;
-      attn_ks = 2;
       const int per_sm = g * B > 64 ? 1 : 2;
       n_splits = std::min(ctx_tiles, std::max(n_splits, (per_sm * ctx->num_sms + pairs - 1) / pairs));
     }
@@ -799,7 +798,12 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
 
   GemmSpec lm;
   lm.x = ctx->h;
-  lm.x_split = ctx->bf16;
+  // The LM head only feeds an argmax: above 32 rows it reads the hi plane alone,
+  // which halves its MMA work and activation tiles (from 64 rows on, the split
+  // makes it tensor- or shared-memory-bound). The hi plane's rounding (2^-9
+  // relative) moves a logit by ~2e-3 (std) at these scales, inside the 1e-2
+  // top-2 gap the draft tokens are held to; up to 32 rows the lo plane is free.
+  lm.x_split = ctx->bf16 && R <= 32;
   lm.ldx = H;
   lm.M = R;
   lm.K = H;
