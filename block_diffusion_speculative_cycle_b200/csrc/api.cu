@@ -167,8 +167,11 @@ struct GemmSpec {
 // the grid within split_slots CTAs per SM (default two), so every CTA streams
 // from the start and a third slot per SM stays free for the next kernel's CTAs
 // to start and prefetch their weights (programmatic dependent launch).
-int choose_splits(dflash_ctx* ctx, int units, int num_kb) {
-  const int slots = ctx->split_slots * ctx->num_sms;
+int choose_splits(dflash_ctx* ctx, int units, int num_kb, int m_tile) {
+  // CTAs of this shape that fit per SM (the ring budgets below: 74 KB up to 32
+  // activation rows, 110 KB up to 64, about 220 KB above)
+  const int fit = m_tile <= 32 ? 3 : (m_tile <= 64 ? 2 : 1);
+  const int slots = std::min(ctx->split_slots, fit) * ctx->num_sms;
   for (int s = kMaxClusterSplits; s >= 2; --s)
     if (num_kb / s >= 2 && units * s <= slots) return s;
   return 1;
@@ -242,7 +245,7 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   p.n_tiles = n_tiles;
   const int units = n_tiles * p.m_blocks;
   p.splits = ctx->force_splits > 0 ? std::min(ctx->force_splits, std::max(1, p.num_kb / 2))
-                                   : choose_splits(ctx, units, p.num_kb);
+                                   : choose_splits(ctx, units, p.num_kb, p.m_tile);
   // ring depth: while m_tile <= 32 keep each CTA (ring + receive buffer) within a
   // third of the SM's shared memory, so three CTAs fit; otherwise use what fits.
   // The split epilogue reuses the ring for this split's rows (m_tile x 128 fp32)
