@@ -642,21 +642,13 @@ static cudaError_t launch_cluster_t(const AttnParams& p, void* out, cudaStream_t
 
 cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {
   if (p.n_splits < 1 || (!p.global_merge && p.n_splits > kMaxAttnCluster) || p.kps % kKT) return cudaErrorInvalidValue;
-  // ks = 1: one warp per 16 query rows; two CTAs fit per SM by registers and
-  // shared memory, which keeps the clusters placeable all at once.
-  // ks = 2 (small grids): two warps per 16 rows, each taking half of every key
-  // tile, and a two-stage ring.
-  const bool wide = p.g * p.B > 64;
-  if (p.ks == 2) {
-    // d = 64: a three-stage ring when a CTA streams more than two tiles (two CTAs
-    // per SM still fit); d = 128 keeps two stages (a third would leave one CTA per SM)
-    if (p.d == 128) return launch_cluster_t<128, 2, 2>(p, out, st, pdl);
-    const bool deep = !wide && p.kps / kKT > 2;
-    return deep ? launch_cluster_t<64, 3, 2>(p, out, st, pdl) : launch_cluster_t<64, 2, 2>(p, out, st, pdl);
-  }
-  if (p.d == 128)
-    return wide ? launch_cluster_t<128, 2, 1>(p, out, st, pdl) : launch_cluster_t<128, 3, 1>(p, out, st, pdl);
-  return wide ? launch_cluster_t<64, 2, 1>(p, out, st, pdl) : launch_cluster_t<64, 3, 1>(p, out, st, pdl);
+  // Two key groups per CTA (every launch): two warps per 16 query rows, each
+  // taking half of every key tile; a two-stage ring (three at d = 64 and <= 64
+  // rows when a CTA streams more than two tiles: two CTAs per SM still fit).
+  if (p.ks != 2) return cudaErrorInvalidValue;
+  if (p.d == 128) return launch_cluster_t<128, 2, 2>(p, out, st, pdl);
+  const bool three = p.g * p.B <= 64 && p.kps / kKT > 2;
+  return three ? launch_cluster_t<64, 3, 2>(p, out, st, pdl) : launch_cluster_t<64, 2, 2>(p, out, st, pdl);
 }
 
 }  // namespace dfl
