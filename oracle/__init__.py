@@ -10,6 +10,8 @@ Modules
   dflash  -- feature fusion + KV injection, the block drafter, greedy verify
   target  -- a tiny causal target model, greedy autoregressive decoding and the
              speculative loop (for the lossless check)
+  sampling -- sampled (temperature > 0) verification and Gumbel-max drafting,
+             the groundwork for the sampled-verify kernel (no CUDA counterpart yet)
 
 Parity status per function (what pins each one, see tests/test_oracle_*.py):
   rms_norm, silu, apply_rope, block_attention, drafter_layer, inject,
@@ -17,4 +19,8 @@ Parity status per function (what pins each one, see tests/test_oracle_*.py):
   greedy_argmax, verify       pinned (brute force, hand-worked golden cases)
   TinyTarget, greedy_decode,
   spec_generate               pinned (library decoder, lossless invariant)
+  softmax_t, sample_index,
+  sampled_verify,
+  gumbel_sample               pinned (exact first-token marginal, special cases,
+                              greedy limit, Markov-chain loop, softmax frequencies)
 """
