@@ -1,9 +1,12 @@
 // Tensor-core block attention (fp16 operands, fp32 accumulate) for the bf16 drafter.
 //
 // One CTA per (split of the key range, KV head, request); the splits of one
-// (request, KV head) form a thread-block cluster. The g*B block queries
-// of the head group (g = n_q/n_kv query heads x B block rows, <= 128 rows) are
-// split into 16-row slices, one per warp, held as mma.sync A fragments. Keys
+// (request, KV head) form a thread-block cluster, or, for long contexts with few
+// (request, KV head) pairs, write their partials to global memory for a merge
+// kernel. The g*B block queries of the head group (g = n_q/n_kv query heads x B
+// block rows, <= 128 rows) are split into 16-row slices; each slice has two warps
+// (key groups), each taking half of every key tile, with the Q fragments read
+// from shared memory for the mma.sync A operand. Keys
 // stream through shared memory in tiles of 64 (a ring of 2-3 stages, cp.async 16-byte
 // copies, XOR-swizzled rows so ldmatrix is conflict-free): context keys come
 // from the request's cache pages, the B block keys from the block K/V rows
@@ -19,7 +22,9 @@
 // those rows (distributed shared memory, counted on that CTA's mbarrier); each
 // owner waits for exactly its rows, combines the splits (log-sum-exp weights,
 // split order) and writes them as a pair of bf16 planes (hi, and lo = the
-// rounding residue out_plane elements further on).
+// rounding residue out_plane elements further on). The launcher instantiates
+// KS = 2 only; the KS = 1 form (one warp per slice, Q held in registers) is kept
+// in the template for reference and measurement.
 #include "kernels.cuh"
 #include "sm100.cuh"
 
