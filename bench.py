@@ -114,30 +114,43 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def setup_dist():
+def setup_dist(backend=None):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE): NCCL when
+    CUDA is present, gloo otherwise (the host-only tests of the replica logic)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The slowest rank's time: every rank's number is device-timed, the job's is the max."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, steps: int, ms_max: float) -> float:
+    """Whole-job cycles/s: every rank runs `steps` cycles of its own replica in ms_max."""
+    return world * steps / (ms_max / 1000.0)
 
 
 def barrier(world):
@@ -386,7 +399,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     ms = ev0.elapsed_time(ev1)
     ms_max = max_over_ranks(ms, world)
-    value = world * args.steps / (ms_max / 1000.0)
+    value = job_throughput(world, args.steps, ms_max)
     clk = clocks.summary()
     c.drafter.check()
 
@@ -508,7 +521,7 @@ def run_ours(args, world, rank, local):
     e1.record(comp)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * e2e_steps / (e2e_ms / 1000.0)
+    e2e_value = job_throughput(world, e2e_steps, e2e_ms)
     h2d = h_feats.numel() * h_feats.element_size() + h_logits.numel() * h_logits.element_size() + h_small.numel() * 4
     d2h = c.bs * (2 + max(c.B - 1, 1)) * 4
     c.drafter.check()
