@@ -11,6 +11,7 @@
 
 #include "../../include/dflash.h"
 #include "gemm.cuh"
+#include "trace.h"
 #include "kernels.cuh"
 
 using namespace dfl;
@@ -512,6 +513,7 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
                                            const int* d_n_new, const int* d_start_pos, void* const* k_cache,
                                            void* const* v_cache, const int* d_page_table, int max_pages,
                                            int num_pages, void* stream) {
+  dfl::TraceRange trace_("dflash_inject_ctx");
   if (!ctx) return DFLASH_ERR_ARG;
   const dflash_config& c = ctx->cfg;
   if (bs <= 0 || bs > c.max_batch || max_new < 0 || (long long)bs * max_new > c.max_inject_rows)
@@ -583,6 +585,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
                                             int B, const void* const* k_cache, const void* const* v_cache,
                                             const int* d_page_table, int max_pages, int num_pages, int max_ctx,
                                             int* d_draft, float* d_hidden_out, void* stream) {
+  dfl::TraceRange trace_("dflash_draft_block");
   if (!ctx) return DFLASH_ERR_ARG;
   const dflash_config& c = ctx->cfg;
   if (bs <= 0 || bs > c.max_batch || B <= 0 || B > c.max_block || max_ctx < 0) return DFLASH_ERR_ARG;

@@ -7,6 +7,7 @@
 // draft[i-1] against argmax row i-1, next = argmax row a; it then zeroes the
 // request's keys and ticket so the workspace is ready for the next call.
 #include <cstdio>
+#include "trace.h"
 #include <cstdlib>
 #include <mutex>
 
@@ -138,6 +139,7 @@ extern "C" size_t dflash_verify_workspace_size(int bs, int B) {
 extern "C" dflash_status dflash_verify(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft, int bs,
                                        int B, int V, int* d_accepted, int* d_next_token, void* d_workspace,
                                        size_t workspace_bytes, void* stream) {
+  dfl::TraceRange trace_("dflash_verify");
   if (bs <= 0 || B <= 0 || V <= 0 || !d_logits || !d_accepted || !d_next_token || !d_workspace) return DFLASH_ERR_ARG;
   if (B > 1 && !d_draft) return DFLASH_ERR_ARG;
   if (logits_dtype != DFLASH_F32 && logits_dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
@@ -188,6 +190,7 @@ cudaError_t noalloc_scratch(void** out) {
 extern "C" dflash_status dflash_verify_noalloc(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft,
                                                int bs, int B, int V, int* d_accepted, int* d_next_token,
                                                void* stream) {
+  dfl::TraceRange trace_("dflash_verify_noalloc");
   if (bs <= 0 || B <= 0 || V <= 0 || !d_logits || !d_accepted || !d_next_token) return DFLASH_ERR_ARG;
   if (B > 1 && !d_draft) return DFLASH_ERR_ARG;
   if (logits_dtype != DFLASH_F32 && logits_dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
