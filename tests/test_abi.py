@@ -70,3 +70,62 @@ def test_drafter_config_marshalling(monkeypatch):
     c = seen.pop("c")
     assert c.dtype == _binding.DFLASH_BF16 and c.cache_dtype == _binding.DFLASH_F16
     assert d.cache_dtype == torch.float16
+
+
+def _valid_config():
+    """A supported bf16 drafter shape (the checks below each break one field)."""
+    c = _binding.dflash_config()
+    c.hidden, c.n_layers, c.n_q_heads, c.n_kv_heads, c.head_dim = 512, 2, 4, 2, 128
+    c.intermediate, c.vocab, c.n_feat_layers, c.target_hidden, c.mask_token_id = 1024, 2048, 3, 256, 2047
+    c.max_block, c.max_batch, c.max_inject_rows, c.page_size = 16, 2, 64, 64
+    c.rope_theta, c.rms_eps, c.dtype, c.cache_dtype = 1e4, 1e-6, _binding.DFLASH_BF16, _binding.DFLASH_BF16
+    return c
+
+
+def _fake_weights():
+    import ctypes
+    w = _binding.dflash_weights()
+    arr = (ctypes.c_void_p * 2)(16, 16)
+    w.fc = w.embed = w.lm_head = w.final_norm = 16   # never dereferenced: every case below fails first
+    for k in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "wgate", "wup", "wdown"):
+        setattr(w, k, ctypes.cast(arr, _binding._PP))
+    return w, arr
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("mask_token_id", 2048, 1),            # outside the vocabulary
+    ("n_kv_heads", 3, 1),                  # n_q not a multiple of n_kv
+    ("dtype", 7, 1),                       # unknown weight type
+    ("head_dim", 96, 6),                   # only 64 and 128
+    ("hidden", 576, 6),                    # not a multiple of the 128-row weight tile
+    ("vocab", 2000, 6),
+    ("max_block", 70, 6),                  # g * B > 128 query rows per head group
+])
+def test_create_validates_each_field_on_the_host(lib_path, field, value, status):
+    import ctypes
+    lib = _binding.load_library(lib_path)
+    c = _valid_config()
+    setattr(c, field, value)
+    if field == "vocab":
+        c.mask_token_id = value - 1
+    w, _keep = _fake_weights()
+    h = ctypes.c_void_p()
+    assert lib.dflash_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == status
+    assert not h.value
+
+
+def test_fp16_cache_needs_a_bf16_drafter(lib_path):
+    import ctypes
+    lib = _binding.load_library(lib_path)
+    c = _valid_config()
+    c.dtype, c.cache_dtype = _binding.DFLASH_F32, _binding.DFLASH_F16
+    w, _keep = _fake_weights()
+    h = ctypes.c_void_p()
+    assert lib.dflash_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == 1
+
+
+def test_cycle_calls_reject_a_null_context(lib_path):
+    lib = _binding.load_library(lib_path)
+    assert lib.dflash_inject_ctx(None, None, 1, 1, None, None, None, None, None, 1, 1, None) == 1
+    assert lib.dflash_draft_block(None, None, None, 1, 4, None, None, None, 1, 1, 0, None, None, None) == 1
+    assert lib.dflash_get_error(None, None) == 1
