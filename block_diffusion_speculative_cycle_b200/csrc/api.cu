@@ -308,151 +308,155 @@ extern "C" const char* dflash_status_string(dflash_status s) {
 }
 
 extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_weights* w, dflash_ctx** out) {
-  if (!cfg || !w || !out) return DFLASH_ERR_ARG;
-  *out = nullptr;
-  const dflash_config& c = *cfg;
-  if (c.hidden <= 0 || c.n_layers < 0 || c.n_q_heads <= 0 || c.n_kv_heads <= 0 || c.head_dim <= 0 ||
-      c.intermediate <= 0 || c.vocab <= 1 || c.n_feat_layers <= 0 || c.target_hidden <= 0 || c.max_block <= 0 ||
-      c.max_batch <= 0 || c.max_inject_rows < 0 || c.page_size <= 0 || !(c.rope_theta > 0.f) || !(c.rms_eps >= 0.f))
-    return DFLASH_ERR_ARG;
-  if (c.mask_token_id < 0 || c.mask_token_id >= c.vocab) return DFLASH_ERR_ARG;
-  if (c.n_q_heads % c.n_kv_heads) return DFLASH_ERR_ARG;
-  if (c.dtype != DFLASH_F32 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
-  if (c.cache_dtype == DFLASH_F16 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
-  if (!w->fc || !w->embed || !w->lm_head || !w->final_norm) return DFLASH_ERR_ARG;
-  if (c.n_layers > 0 && (!w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo || !w->mlp_norm || !w->wgate ||
-                         !w->wup || !w->wdown))
-    return DFLASH_ERR_ARG;
-  // shape support: 128-row weight tiles aligned to segment starts, paired 64-row gate/up tiles
-  const int F = c.n_feat_layers * c.target_hidden;
-  const int kalign = c.dtype == DFLASH_BF16 ? 64 : 32;
-  if (c.head_dim != 64 && c.head_dim != 128) return DFLASH_ERR_UNSUPPORTED;
-  if (c.hidden % 128 || q_dim(c) % 128 || kv_dim(c) % 128 || c.intermediate % 64 || c.vocab % 128)
-    return DFLASH_ERR_UNSUPPORTED;
-  if (c.hidden % kalign || q_dim(c) % kalign || c.intermediate % kalign || F % kalign) return DFLASH_ERR_UNSUPPORTED;
-  if ((c.n_q_heads / c.n_kv_heads) * c.max_block > 128) return DFLASH_ERR_UNSUPPORTED;
-
-  dflash_ctx* ctx = new dflash_ctx();
-  ctx->cfg = c;
-  ctx->bf16 = c.dtype == DFLASH_BF16;
-  ctx->cache_f16 = c.cache_dtype == DFLASH_F16;
-  const char* env = std::getenv("DFLASH_FORCE_SIMT");
-  ctx->force_simt = env && env[0] == '1';
-  env = std::getenv("DFLASH_DEBUG");
-  ctx->debug = env && env[0] == '1';
-  env = std::getenv("DFLASH_SPLITS");
-  ctx->force_splits = env ? std::atoi(env) : 0;
-  if (ctx->force_splits > kMaxClusterSplits) ctx->force_splits = kMaxClusterSplits;
-  env = std::getenv("DFLASH_SPLIT_SLOTS");
-  if (env && std::atoi(env) >= 1 && std::atoi(env) <= 3) ctx->split_slots = std::atoi(env);
-  env = std::getenv("DFLASH_STAGES");
-  ctx->force_stages = env ? std::atoi(env) : 0;
-  if (ctx->force_stages > 8) ctx->force_stages = 8;
-  env = std::getenv("DFLASH_PDL");
-  ctx->use_pdl = !(env && env[0] == '0');
-  int dev = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev);
-  ctx->fc = w->fc;
-  ctx->embed = w->embed;
-  ctx->lm_head = w->lm_head;
-  ctx->final_norm = w->final_norm;
-  for (int l = 0; l < c.n_layers; ++l) {
-    if (!w->attn_norm[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->mlp_norm[l] || !w->wgate[l] ||
-        !w->wup[l] || !w->wdown[l]) {
-      delete ctx;
+  try {
+    if (!cfg || !w || !out) return DFLASH_ERR_ARG;
+    *out = nullptr;
+    const dflash_config& c = *cfg;
+    if (c.hidden <= 0 || c.n_layers < 0 || c.n_q_heads <= 0 || c.n_kv_heads <= 0 || c.head_dim <= 0 ||
+        c.intermediate <= 0 || c.vocab <= 1 || c.n_feat_layers <= 0 || c.target_hidden <= 0 || c.max_block <= 0 ||
+        c.max_batch <= 0 || c.max_inject_rows < 0 || c.page_size <= 0 || !(c.rope_theta > 0.f) || !(c.rms_eps >= 0.f))
       return DFLASH_ERR_ARG;
+    if (c.mask_token_id < 0 || c.mask_token_id >= c.vocab) return DFLASH_ERR_ARG;
+    if (c.n_q_heads % c.n_kv_heads) return DFLASH_ERR_ARG;
+    if (c.dtype != DFLASH_F32 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
+    if (c.cache_dtype == DFLASH_F16 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
+    if (!w->fc || !w->embed || !w->lm_head || !w->final_norm) return DFLASH_ERR_ARG;
+    if (c.n_layers > 0 && (!w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo || !w->mlp_norm || !w->wgate ||
+                           !w->wup || !w->wdown))
+      return DFLASH_ERR_ARG;
+    // shape support: 128-row weight tiles aligned to segment starts, paired 64-row gate/up tiles
+    const int F = c.n_feat_layers * c.target_hidden;
+    const int kalign = c.dtype == DFLASH_BF16 ? 64 : 32;
+    if (c.head_dim != 64 && c.head_dim != 128) return DFLASH_ERR_UNSUPPORTED;
+    if (c.hidden % 128 || q_dim(c) % 128 || kv_dim(c) % 128 || c.intermediate % 64 || c.vocab % 128)
+      return DFLASH_ERR_UNSUPPORTED;
+    if (c.hidden % kalign || q_dim(c) % kalign || c.intermediate % kalign || F % kalign) return DFLASH_ERR_UNSUPPORTED;
+    if ((c.n_q_heads / c.n_kv_heads) * c.max_block > 128) return DFLASH_ERR_UNSUPPORTED;
+
+    dflash_ctx* ctx = new dflash_ctx();
+    ctx->cfg = c;
+    ctx->bf16 = c.dtype == DFLASH_BF16;
+    ctx->cache_f16 = c.cache_dtype == DFLASH_F16;
+    const char* env = std::getenv("DFLASH_FORCE_SIMT");
+    ctx->force_simt = env && env[0] == '1';
+    env = std::getenv("DFLASH_DEBUG");
+    ctx->debug = env && env[0] == '1';
+    env = std::getenv("DFLASH_SPLITS");
+    ctx->force_splits = env ? std::atoi(env) : 0;
+    if (ctx->force_splits > kMaxClusterSplits) ctx->force_splits = kMaxClusterSplits;
+    env = std::getenv("DFLASH_SPLIT_SLOTS");
+    if (env && std::atoi(env) >= 1 && std::atoi(env) <= 3) ctx->split_slots = std::atoi(env);
+    env = std::getenv("DFLASH_STAGES");
+    ctx->force_stages = env ? std::atoi(env) : 0;
+    if (ctx->force_stages > 8) ctx->force_stages = 8;
+    env = std::getenv("DFLASH_PDL");
+    ctx->use_pdl = !(env && env[0] == '0');
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev);
+    ctx->fc = w->fc;
+    ctx->embed = w->embed;
+    ctx->lm_head = w->lm_head;
+    ctx->final_norm = w->final_norm;
+    for (int l = 0; l < c.n_layers; ++l) {
+      if (!w->attn_norm[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->mlp_norm[l] || !w->wgate[l] ||
+          !w->wup[l] || !w->wdown[l]) {
+        delete ctx;
+        return DFLASH_ERR_ARG;
+      }
+      ctx->attn_norm.push_back(w->attn_norm[l]);
+      ctx->mlp_norm.push_back(w->mlp_norm[l]);
+      ctx->wq.push_back(w->wq[l]);
+      ctx->wk.push_back(w->wk[l]);
+      ctx->wv.push_back(w->wv[l]);
+      ctx->wo.push_back(w->wo[l]);
+      ctx->wg.push_back(w->wgate[l]);
+      ctx->wu.push_back(w->wup[l]);
+      ctx->wd.push_back(w->wdown[l]);
     }
-    ctx->attn_norm.push_back(w->attn_norm[l]);
-    ctx->mlp_norm.push_back(w->mlp_norm[l]);
-    ctx->wq.push_back(w->wq[l]);
-    ctx->wk.push_back(w->wk[l]);
-    ctx->wv.push_back(w->wv[l]);
-    ctx->wo.push_back(w->wo[l]);
-    ctx->wg.push_back(w->wgate[l]);
-    ctx->wu.push_back(w->wup[l]);
-    ctx->wd.push_back(w->wdown[l]);
-  }
 
-  cudaDriverEntryPointQueryResult qres;
-  void* fn = nullptr;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
-      qres != cudaDriverEntryPointSuccess || !fn) {
-    delete ctx;
-    return DFLASH_ERR_CUDA;
-  }
-  ctx->encode = reinterpret_cast<EncodeTiledFn>(fn);
+    cudaDriverEntryPointQueryResult qres;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess || !fn) {
+      delete ctx;
+      return DFLASH_ERR_CUDA;
+    }
+    ctx->encode = reinterpret_cast<EncodeTiledFn>(fn);
 
-  // workspace layout
-  const size_t R = (size_t)c.max_batch * c.max_block;
-  const size_t Rin = std::max(1, c.max_inject_rows);
-  const size_t es = esize(ctx);
-  const int g = c.n_q_heads / c.n_kv_heads;
-  const size_t nr = (size_t)g * c.max_block;
-  ctx->att_rows = ((size_t)kAttnTargetCtas + (size_t)c.max_batch * c.n_kv_heads + 8) * nr;
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    size_t o = off;
-    off += align256(bytes);
-    return o;
-  };
-  const size_t o_x = take(R * c.hidden * 4);
-  const size_t planes = ctx->bf16 ? 2 : 1;   // bf16 activations are stored as hi/lo planes
-  const size_t o_h = take(planes * R * c.hidden * es);
-  const size_t o_q = take(R * q_dim(c) * es);
-  const size_t o_kb = take(R * kv_dim(c) * es);
-  const size_t o_vb = take(R * kv_dim(c) * es);
-  const size_t o_ao = take(planes * R * q_dim(c) * es);
-  const size_t o_act = take(planes * R * c.intermediate * es);
-  const size_t o_c = take(planes * Rin * c.hidden * es);
-  const size_t o_keys = take(R * 8);
-  const size_t o_atto = take(ctx->att_rows * c.head_dim * 4);
-  const size_t o_attm = take(ctx->att_rows * 4);
-  const size_t o_attl = take(ctx->att_rows * 4);
-  const size_t o_st = take(256);
-  const size_t o_freq = take((size_t)c.head_dim / 2 * sizeof(double));
-  const size_t o_ss0 = take((size_t)(c.hidden / 128) * R * 4);
-  const size_t o_ss1 = take((size_t)(c.hidden / 128) * R * 4);
-  ctx->ws_bytes = off;
-  if (cudaMalloc(&ctx->ws, off) != cudaSuccess) {
-    cudaGetLastError();
-    delete ctx;
-    return DFLASH_ERR_OOM;
-  }
-  if (cudaMemset(ctx->ws, 0, off) != cudaSuccess) {
-    cudaFree(ctx->ws);
-    delete ctx;
-    return DFLASH_ERR_CUDA;
-  }
-  char* b = ctx->ws;
-  ctx->x = (float*)(b + o_x);
-  ctx->h = b + o_h;
-  ctx->q = b + o_q;
-  ctx->kb = b + o_kb;
-  ctx->vb = b + o_vb;
-  ctx->ao = b + o_ao;
-  ctx->act = b + o_act;
-  ctx->c = b + o_c;
-  ctx->keys = (unsigned long long*)(b + o_keys);
-  ctx->att_o = (float*)(b + o_atto);
-  ctx->att_m = (float*)(b + o_attm);
-  ctx->att_l = (float*)(b + o_attl);
-  ctx->status = (int*)(b + o_st);
-  ctx->inv_freq = (double*)(b + o_freq);
-  ctx->sumsq[0] = (float*)(b + o_ss0);
-  ctx->sumsq[1] = (float*)(b + o_ss1);
-  {
-    // theta^(-2i/d), i = 0..d/2-1, in double
-    std::vector<double> f(c.head_dim / 2);
-    for (int i = 0; i < c.head_dim / 2; ++i) f[i] = std::pow((double)c.rope_theta, -2.0 * i / c.head_dim);
-    if (cudaMemcpy(ctx->inv_freq, f.data(), f.size() * sizeof(double), cudaMemcpyHostToDevice) != cudaSuccess) {
+    // workspace layout
+    const size_t R = (size_t)c.max_batch * c.max_block;
+    const size_t Rin = std::max(1, c.max_inject_rows);
+    const size_t es = esize(ctx);
+    const int g = c.n_q_heads / c.n_kv_heads;
+    const size_t nr = (size_t)g * c.max_block;
+    ctx->att_rows = ((size_t)kAttnTargetCtas + (size_t)c.max_batch * c.n_kv_heads + 8) * nr;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+      size_t o = off;
+      off += align256(bytes);
+      return o;
+    };
+    const size_t o_x = take(R * c.hidden * 4);
+    const size_t planes = ctx->bf16 ? 2 : 1;   // bf16 activations are stored as hi/lo planes
+    const size_t o_h = take(planes * R * c.hidden * es);
+    const size_t o_q = take(R * q_dim(c) * es);
+    const size_t o_kb = take(R * kv_dim(c) * es);
+    const size_t o_vb = take(R * kv_dim(c) * es);
+    const size_t o_ao = take(planes * R * q_dim(c) * es);
+    const size_t o_act = take(planes * R * c.intermediate * es);
+    const size_t o_c = take(planes * Rin * c.hidden * es);
+    const size_t o_keys = take(R * 8);
+    const size_t o_atto = take(ctx->att_rows * c.head_dim * 4);
+    const size_t o_attm = take(ctx->att_rows * 4);
+    const size_t o_attl = take(ctx->att_rows * 4);
+    const size_t o_st = take(256);
+    const size_t o_freq = take((size_t)c.head_dim / 2 * sizeof(double));
+    const size_t o_ss0 = take((size_t)(c.hidden / 128) * R * 4);
+    const size_t o_ss1 = take((size_t)(c.hidden / 128) * R * 4);
+    ctx->ws_bytes = off;
+    if (cudaMalloc(&ctx->ws, off) != cudaSuccess) {
+      cudaGetLastError();
+      delete ctx;
+      return DFLASH_ERR_OOM;
+    }
+    if (cudaMemset(ctx->ws, 0, off) != cudaSuccess) {
       cudaFree(ctx->ws);
       delete ctx;
       return DFLASH_ERR_CUDA;
     }
+    char* b = ctx->ws;
+    ctx->x = (float*)(b + o_x);
+    ctx->h = b + o_h;
+    ctx->q = b + o_q;
+    ctx->kb = b + o_kb;
+    ctx->vb = b + o_vb;
+    ctx->ao = b + o_ao;
+    ctx->act = b + o_act;
+    ctx->c = b + o_c;
+    ctx->keys = (unsigned long long*)(b + o_keys);
+    ctx->att_o = (float*)(b + o_atto);
+    ctx->att_m = (float*)(b + o_attm);
+    ctx->att_l = (float*)(b + o_attl);
+    ctx->status = (int*)(b + o_st);
+    ctx->inv_freq = (double*)(b + o_freq);
+    ctx->sumsq[0] = (float*)(b + o_ss0);
+    ctx->sumsq[1] = (float*)(b + o_ss1);
+    {
+      // theta^(-2i/d), i = 0..d/2-1, in double
+      std::vector<double> f(c.head_dim / 2);
+      for (int i = 0; i < c.head_dim / 2; ++i) f[i] = std::pow((double)c.rope_theta, -2.0 * i / c.head_dim);
+      if (cudaMemcpy(ctx->inv_freq, f.data(), f.size() * sizeof(double), cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaFree(ctx->ws);
+        delete ctx;
+        return DFLASH_ERR_CUDA;
+      }
+    }
+    *out = ctx;
+    return DFLASH_OK;
+  } catch (...) {   // no C++ exception crosses the C ABI
+    return DFLASH_ERR_OOM;
   }
-  *out = ctx;
-  return DFLASH_OK;
 }
 
 extern "C" void dflash_destroy(dflash_ctx* ctx) {
@@ -469,32 +473,36 @@ extern "C" dflash_status dflash_profile_enable(dflash_ctx* ctx, int enable) {
 }
 
 extern "C" int dflash_profile_read(dflash_ctx* ctx, dflash_profile_entry* out, int max_entries) {
-  if (!ctx || (!out && max_entries > 0)) return -(int)DFLASH_ERR_ARG;
-  dflash_profile_entry agg[PK_COUNT];
-  std::memset(agg, 0, sizeof(agg));
-  bool fail = false;
-  for (ProfRec& r : ctx->recs) {
-    float ms = 0.f;
-    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) fail = true;
-    agg[r.kind].launches += 1;
-    agg[r.kind].total_ms += ms;
-    agg[r.kind].bytes += r.bytes;
-    agg[r.kind].flops += r.flops;
-    cudaEventDestroy(r.a);
-    cudaEventDestroy(r.b);
-  }
-  ctx->recs.clear();
-  if (fail) return -(int)DFLASH_ERR_CUDA;
-  int n = 0;
-  for (int k = 0; k < PK_COUNT; ++k) {
-    if (!agg[k].launches) continue;
-    if (n < max_entries) {
-      out[n] = agg[k];
-      std::strncpy(out[n].name, kProfNames[k], sizeof(out[n].name) - 1);
+  try {
+    if (!ctx || (!out && max_entries > 0)) return -(int)DFLASH_ERR_ARG;
+    dflash_profile_entry agg[PK_COUNT];
+    std::memset(agg, 0, sizeof(agg));
+    bool fail = false;
+    for (ProfRec& r : ctx->recs) {
+      float ms = 0.f;
+      if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) fail = true;
+      agg[r.kind].launches += 1;
+      agg[r.kind].total_ms += ms;
+      agg[r.kind].bytes += r.bytes;
+      agg[r.kind].flops += r.flops;
+      cudaEventDestroy(r.a);
+      cudaEventDestroy(r.b);
     }
-    ++n;
+    ctx->recs.clear();
+    if (fail) return -(int)DFLASH_ERR_CUDA;
+    int n = 0;
+    for (int k = 0; k < PK_COUNT; ++k) {
+      if (!agg[k].launches) continue;
+      if (n < max_entries) {
+        out[n] = agg[k];
+        std::strncpy(out[n].name, kProfNames[k], sizeof(out[n].name) - 1);
+      }
+      ++n;
+    }
+    return std::min(n, max_entries);
+  } catch (...) {   // no C++ exception crosses the C ABI
+    return -1;
   }
-  return std::min(n, max_entries);
 }
 
 extern "C" dflash_status dflash_get_error(dflash_ctx* ctx, void* stream) {
@@ -514,71 +522,75 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
                                            void* const* v_cache, const int* d_page_table, int max_pages,
                                            int num_pages, void* stream) {
   dfl::TraceRange trace_("dflash_inject_ctx");
-  if (!ctx) return DFLASH_ERR_ARG;
-  const dflash_config& c = ctx->cfg;
-  if (bs <= 0 || bs > c.max_batch || max_new < 0 || (long long)bs * max_new > c.max_inject_rows)
-    return DFLASH_ERR_ARG;
-  if (max_new == 0) return DFLASH_OK;
-  if (!feats || !d_n_new || !d_start_pos || !d_page_table || max_pages <= 0 || num_pages <= 0) return DFLASH_ERR_ARG;
-  if (c.n_layers > 0 && (!k_cache || !v_cache)) return DFLASH_ERR_ARG;
-  for (int l = 0; l < c.n_layers; ++l)
-    if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_ARG;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int M = bs * max_new;
-  const int F = c.n_feat_layers * c.target_hidden;
+  try {
+    if (!ctx) return DFLASH_ERR_ARG;
+    const dflash_config& c = ctx->cfg;
+    if (bs <= 0 || bs > c.max_batch || max_new < 0 || (long long)bs * max_new > c.max_inject_rows)
+      return DFLASH_ERR_ARG;
+    if (max_new == 0) return DFLASH_OK;
+    if (!feats || !d_n_new || !d_start_pos || !d_page_table || max_pages <= 0 || num_pages <= 0) return DFLASH_ERR_ARG;
+    if (c.n_layers > 0 && (!k_cache || !v_cache)) return DFLASH_ERR_ARG;
+    for (int l = 0; l < c.n_layers; ++l)
+      if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int M = bs * max_new;
+    const int F = c.n_feat_layers * c.target_hidden;
 
-  GemmSpec fcg;
-  fcg.x = feats;
-  fcg.ldx = F;
-  fcg.M = M;
-  fcg.K = F;
-  fcg.n_seg = 1;
-  fcg.w[0] = ctx->fc;
-  fcg.seg_rows[0] = c.hidden;
-  fcg.tag = TAG_FC;
-  fcg.epi.kind = EPI_STORE;
-  fcg.epi.out[0] = ctx->c;
-  fcg.epi.ld_out[0] = c.hidden;
-  fcg.epi.out_type = OUT_BF16X2;   // c feeds the K/V GEMM as hi/lo planes
-  fcg.epi.out_plane = (size_t)M * c.hidden;
-  fcg.epi.rows_per_req = max_new;
-  DFL_CHECK(run_gemm(ctx, fcg, st));
+    GemmSpec fcg;
+    fcg.x = feats;
+    fcg.ldx = F;
+    fcg.M = M;
+    fcg.K = F;
+    fcg.n_seg = 1;
+    fcg.w[0] = ctx->fc;
+    fcg.seg_rows[0] = c.hidden;
+    fcg.tag = TAG_FC;
+    fcg.epi.kind = EPI_STORE;
+    fcg.epi.out[0] = ctx->c;
+    fcg.epi.ld_out[0] = c.hidden;
+    fcg.epi.out_type = OUT_BF16X2;   // c feeds the K/V GEMM as hi/lo planes
+    fcg.epi.out_plane = (size_t)M * c.hidden;
+    fcg.epi.rows_per_req = max_new;
+    DFL_CHECK(run_gemm(ctx, fcg, st));
 
-  // all layers' K and V projections of c, up to kMaxSeg segments per launch
-  const int per_launch = kMaxSeg / 2;
-  for (int l0 = 0, part = 0; l0 < c.n_layers; l0 += per_launch, ++part) {
-    const int nl = std::min(per_launch, c.n_layers - l0);
-    GemmSpec kv;
-    kv.x = ctx->c;
-    kv.x_split = ctx->bf16;
-    kv.ldx = c.hidden;
-    kv.M = M;
-    kv.K = c.hidden;
-    kv.n_seg = 2 * nl;
-    kv.tag = TAG_KV;
-    EpiParams& e = kv.epi;
-    e.kind = EPI_KV_INJECT;
-    for (int i = 0; i < nl; ++i) {
-      kv.w[2 * i] = ctx->wk[l0 + i];
-      kv.w[2 * i + 1] = ctx->wv[l0 + i];
-      kv.seg_rows[2 * i] = kv.seg_rows[2 * i + 1] = kv_dim(c);
-      e.out[2 * i] = k_cache[l0 + i];
-      e.out[2 * i + 1] = v_cache[l0 + i];
-      e.rope_mask |= 1u << (2 * i);
+    // all layers' K and V projections of c, up to kMaxSeg segments per launch
+    const int per_launch = kMaxSeg / 2;
+    for (int l0 = 0, part = 0; l0 < c.n_layers; l0 += per_launch, ++part) {
+      const int nl = std::min(per_launch, c.n_layers - l0);
+      GemmSpec kv;
+      kv.x = ctx->c;
+      kv.x_split = ctx->bf16;
+      kv.ldx = c.hidden;
+      kv.M = M;
+      kv.K = c.hidden;
+      kv.n_seg = 2 * nl;
+      kv.tag = TAG_KV;
+      EpiParams& e = kv.epi;
+      e.kind = EPI_KV_INJECT;
+      for (int i = 0; i < nl; ++i) {
+        kv.w[2 * i] = ctx->wk[l0 + i];
+        kv.w[2 * i + 1] = ctx->wv[l0 + i];
+        kv.seg_rows[2 * i] = kv.seg_rows[2 * i + 1] = kv_dim(c);
+        e.out[2 * i] = k_cache[l0 + i];
+        e.out[2 * i + 1] = v_cache[l0 + i];
+        e.rope_mask |= 1u << (2 * i);
+      }
+      e.head_dim = c.head_dim;
+      e.inv_freq = ctx->inv_freq;
+      e.rows_per_req = max_new;
+      e.pos_base = d_start_pos;
+      e.row_count = d_n_new;
+      e.page_table = d_page_table;
+      e.max_pages = max_pages;
+      e.num_pages = num_pages;
+      e.page_size = c.page_size;
+      e.n_kv = c.n_kv_heads;
+      DFL_CHECK(run_gemm(ctx, kv, st));
     }
-    e.head_dim = c.head_dim;
-    e.inv_freq = ctx->inv_freq;
-    e.rows_per_req = max_new;
-    e.pos_base = d_start_pos;
-    e.row_count = d_n_new;
-    e.page_table = d_page_table;
-    e.max_pages = max_pages;
-    e.num_pages = num_pages;
-    e.page_size = c.page_size;
-    e.n_kv = c.n_kv_heads;
-    DFL_CHECK(run_gemm(ctx, kv, st));
+    return DFLASH_OK;
+  } catch (...) {   // no C++ exception crosses the C ABI
+    return DFLASH_ERR_OOM;
   }
-  return DFLASH_OK;
 }
 
 extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_len, int bs,
@@ -586,245 +598,249 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
                                             const int* d_page_table, int max_pages, int num_pages, int max_ctx,
                                             int* d_draft, float* d_hidden_out, void* stream) {
   dfl::TraceRange trace_("dflash_draft_block");
-  if (!ctx) return DFLASH_ERR_ARG;
-  const dflash_config& c = ctx->cfg;
-  if (bs <= 0 || bs > c.max_batch || B <= 0 || B > c.max_block || max_ctx < 0) return DFLASH_ERR_ARG;
-  if (!d_anchor || !d_ctx_len || (B > 1 && !d_draft)) return DFLASH_ERR_ARG;
-  if (c.n_layers > 0 && (!k_cache || !v_cache)) return DFLASH_ERR_ARG;
-  for (int l = 0; l < c.n_layers; ++l)
-    if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_ARG;
-  if (max_ctx > 0 && (!d_page_table || max_pages <= 0 || num_pages <= 0)) return DFLASH_ERR_ARG;
-  if (max_ctx > (long long)max_pages * c.page_size) return DFLASH_ERR_ARG;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int R = bs * B;
-  const int H = c.hidden, QD = q_dim(c), KVD = kv_dim(c);
-  const int hb = ctx->bf16 ? 1 : 0;
-  const size_t layer_stride = (size_t)R * H;
+  try {
+    if (!ctx) return DFLASH_ERR_ARG;
+    const dflash_config& c = ctx->cfg;
+    if (bs <= 0 || bs > c.max_batch || B <= 0 || B > c.max_block || max_ctx < 0) return DFLASH_ERR_ARG;
+    if (!d_anchor || !d_ctx_len || (B > 1 && !d_draft)) return DFLASH_ERR_ARG;
+    if (c.n_layers > 0 && (!k_cache || !v_cache)) return DFLASH_ERR_ARG;
+    for (int l = 0; l < c.n_layers; ++l)
+      if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_ARG;
+    if (max_ctx > 0 && (!d_page_table || max_pages <= 0 || num_pages <= 0)) return DFLASH_ERR_ARG;
+    if (max_ctx > (long long)max_pages * c.page_size) return DFLASH_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int R = bs * B;
+    const int H = c.hidden, QD = q_dim(c), KVD = kv_dim(c);
+    const int hb = ctx->bf16 ? 1 : 0;
+    const size_t layer_stride = (size_t)R * H;
 
-  const double es = (double)esize(ctx);
-  {
-    ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
-    DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, B, R, c.vocab, H,
-                                            c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps,
-                                            ctx->x, ctx->h, hb, hb ? (size_t)R * H : 0, ctx->status, st,
-                                            ctx->use_pdl),
-                          "embed_norm launch"));
-  }
-  const double norm_bytes = (double)R * H * (4 + es);
-
-  // attention split plan. The context of the longest request is cut into n_splits
-  // ranges of kps keys (a multiple of the kernel's key tile); the last range also
-  // takes the B block keys. Tensor-core path: the splits of one (request, KV head)
-  // form a cluster (<= 16) and merge through distributed shared memory. With few
-  // (request, KV head) pairs and <= 64 query rows the kernel runs two key groups
-  // per CTA and one wave of CTAs (one per SM); otherwise one key group and about
-  // two CTAs per SM. Long contexts get enough splits for <= kAttnTilesPerCta key
-  // tiles per CTA; when 16 splits leave both the GPU under-filled and the CTAs
-  // long, the splits write their partials to global memory and a second kernel
-  // merges them (any split count).
-  const int g = c.n_q_heads / c.n_kv_heads;
-  const int pairs = bs * c.n_kv_heads;
-  const int key_tile = ctx->bf16 ? 64 : 32;
-  const int ctx_tiles = std::max(1, (max_ctx + key_tile - 1) / key_tile);
-  int attn_ks = 1, n_splits;
-  bool attn_gmerge = false;
-  if (ctx->bf16) {
-    const bool small = g * B <= 64 && ctx->num_sms / pairs >= 8;
-    const int want = small ? ctx->num_sms / pairs : (kAttnTargetCtas + pairs - 1) / pairs;
-    n_splits = std::min(want, kMaxAttnCluster);
-    attn_ks = 2;   // two key groups per CTA (two CTAs per SM at <= 64 query rows, one at 128)
-    if ((ctx_tiles + n_splits - 1) / n_splits > kAttnTilesPerCta && pairs * kMaxAttnCluster < kAttnTargetCtas) {
-      // long context, few pairs: one wave of two-group CTAs (one per SM at 128
-      // query rows, two at <= 64), partials merged by a second kernel
-      attn_gmerge = true;
-      const int per_sm = g * B > 64 ? 1 : 2;
-      n_splits = std::min(ctx_tiles, std::max(n_splits, (per_sm * ctx->num_sms + pairs - 1) / pairs));
-    }
-  } else {
-    n_splits = std::max(1, (kAttnTargetCtas + pairs - 1) / pairs);
-  }
-  int kps = (std::max(max_ctx, 1) + n_splits - 1) / n_splits;
-  kps = (kps + key_tile - 1) / key_tile * key_tile;
-  n_splits = std::max(1, (max_ctx + kps - 1) / kps);
-  // split partials in global memory (CUDA-core path, or the global merge) must fit the workspace
-  if ((!ctx->bf16 || attn_gmerge) && (size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows)
-    return DFLASH_ERR_UNSUPPORTED;
-
-  for (int l = 0; l < c.n_layers; ++l) {
-    GemmSpec qkv;
-    qkv.x = ctx->h;
-    qkv.x_split = ctx->bf16;
-    qkv.ldx = H;
-    qkv.M = R;
-    qkv.K = H;
-    qkv.n_seg = 3;
-    qkv.w[0] = ctx->wq[l];
-    qkv.w[1] = ctx->wk[l];
-    qkv.w[2] = ctx->wv[l];
-    qkv.seg_rows[0] = QD;
-    qkv.seg_rows[1] = KVD;
-    qkv.seg_rows[2] = KVD;
-    qkv.tag = TAG_QKV;
-    qkv.epi.kind = EPI_QKV;
-    qkv.epi.out_type = OUT_F16;   // the attention kernel runs in fp16
-    qkv.epi.out[0] = ctx->q;
-    qkv.epi.out[1] = ctx->kb;
-    qkv.epi.out[2] = ctx->vb;
-    qkv.epi.ld_out[0] = QD;
-    qkv.epi.ld_out[1] = KVD;
-    qkv.epi.ld_out[2] = KVD;
-    qkv.epi.rope_mask = 3u;
-    qkv.epi.head_dim = c.head_dim;
-    qkv.epi.inv_freq = ctx->inv_freq;
-    qkv.epi.rows_per_req = B;
-    qkv.epi.pos_base = d_ctx_len;
-    if (l > 0) set_deferred_norm(ctx, qkv.epi, ctx->sumsq[1], R);   // rows carry the previous layer's norm
-    DFL_CHECK(run_gemm(ctx, qkv, st));
-
-    AttnParams ap{};
-    ap.q = ctx->q;
-    ap.kblk = ctx->kb;
-    ap.vblk = ctx->vb;
-    ap.kc = k_cache[l];
-    ap.vc = v_cache[l];
-    ap.ctx_len = d_ctx_len;
-    ap.page_table = d_page_table;
-    ap.max_pages = max_pages;
-    ap.num_pages = num_pages;
-    ap.page_size = c.page_size;
-    ap.bs = bs;
-    ap.B = B;
-    ap.n_q = c.n_q_heads;
-    ap.n_kv = c.n_kv_heads;
-    ap.d = c.head_dim;
-    ap.g = g;
-    ap.kps = kps;
-    ap.n_splits = n_splits;
-    ap.ks = attn_ks;
-    ap.global_merge = attn_gmerge ? 1 : 0;
-    ap.max_ctx = max_ctx;
-    ap.scale = (float)(1.0 / std::sqrt((double)c.head_dim));
-    ap.part_o = ctx->att_o;
-    ap.part_m = ctx->att_m;
-    ap.part_l = ctx->att_l;
-    ap.status = ctx->status;
-    ap.out_plane = (size_t)R * QD;
-    ap.cache_f16 = ctx->cache_f16 ? 1 : 0;
+    const double es = (double)esize(ctx);
     {
-      // context K/V of every request (upper bound max_ctx), block q/k/v, output
-      const double kvb = (double)bs * max_ctx * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;
-      const double fl = 4.0 * bs * B * (double)(max_ctx + B) * QD;
-      ProfScope prof(ctx, PK_ATTN, st, kvb, fl);
-      DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, hb, hb, st, ctx->use_pdl), "attention launch"));
+      ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
+      DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, B, R, c.vocab, H,
+                                              c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps,
+                                              ctx->x, ctx->h, hb, hb ? (size_t)R * H : 0, ctx->status, st,
+                                              ctx->use_pdl),
+                            "embed_norm launch"));
     }
+    const double norm_bytes = (double)R * H * (4 + es);
 
-    GemmSpec o;
-    o.x = ctx->ao;
-    o.x_split = ctx->bf16;
-    o.ldx = QD;
-    o.M = R;
-    o.K = QD;
-    o.n_seg = 1;
-    o.w[0] = ctx->wo[l];
-    o.seg_rows[0] = H;
-    o.tag = TAG_O;
-    o.epi.kind = EPI_RESID;
-    o.epi.x = ctx->x;
-    o.epi.ldx = H;
-    // the MLP norm is deferred: x ⊙ gain now, the row scales in the gate/up epilogue
-    o.epi.gamma_next = ctx->mlp_norm[l];
-    o.epi.out_type = OUT_BF16X2;
-    o.epi.out_plane = (size_t)R * H;
-    o.epi.xg = ctx->h;
-    o.epi.sumsq = ctx->sumsq[0];
-    o.epi.ld_part = R;
-    DFL_CHECK(run_gemm(ctx, o, st));
+    // attention split plan. The context of the longest request is cut into n_splits
+    // ranges of kps keys (a multiple of the kernel's key tile); the last range also
+    // takes the B block keys. Tensor-core path: the splits of one (request, KV head)
+    // form a cluster (<= 16) and merge through distributed shared memory. With few
+    // (request, KV head) pairs and <= 64 query rows the kernel runs two key groups
+    // per CTA and one wave of CTAs (one per SM); otherwise one key group and about
+    // two CTAs per SM. Long contexts get enough splits for <= kAttnTilesPerCta key
+    // tiles per CTA; when 16 splits leave both the GPU under-filled and the CTAs
+    // long, the splits write their partials to global memory and a second kernel
+    // merges them (any split count).
+    const int g = c.n_q_heads / c.n_kv_heads;
+    const int pairs = bs * c.n_kv_heads;
+    const int key_tile = ctx->bf16 ? 64 : 32;
+    const int ctx_tiles = std::max(1, (max_ctx + key_tile - 1) / key_tile);
+    int attn_ks = 1, n_splits;
+    bool attn_gmerge = false;
+    if (ctx->bf16) {
+      const bool small = g * B <= 64 && ctx->num_sms / pairs >= 8;
+      const int want = small ? ctx->num_sms / pairs : (kAttnTargetCtas + pairs - 1) / pairs;
+      n_splits = std::min(want, kMaxAttnCluster);
+      attn_ks = 2;   // two key groups per CTA (two CTAs per SM at <= 64 query rows, one at 128)
+      if ((ctx_tiles + n_splits - 1) / n_splits > kAttnTilesPerCta && pairs * kMaxAttnCluster < kAttnTargetCtas) {
+        // long context, few pairs: one wave of two-group CTAs (one per SM at 128
+        // query rows, two at <= 64), partials merged by a second kernel
+        attn_gmerge = true;
+        const int per_sm = g * B > 64 ? 1 : 2;
+        n_splits = std::min(ctx_tiles, std::max(n_splits, (per_sm * ctx->num_sms + pairs - 1) / pairs));
+      }
+    } else {
+      n_splits = std::max(1, (kAttnTargetCtas + pairs - 1) / pairs);
+    }
+    int kps = (std::max(max_ctx, 1) + n_splits - 1) / n_splits;
+    kps = (kps + key_tile - 1) / key_tile * key_tile;
+    n_splits = std::max(1, (max_ctx + kps - 1) / kps);
+    // split partials in global memory (CUDA-core path, or the global merge) must fit the workspace
+    if ((!ctx->bf16 || attn_gmerge) && (size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows)
+      return DFLASH_ERR_UNSUPPORTED;
 
-    GemmSpec gu;
-    gu.x = ctx->h;
-    gu.x_split = ctx->bf16;
-    gu.ldx = H;
-    gu.M = R;
-    gu.K = H;
-    gu.n_seg = 2;
-    gu.paired = true;
-    gu.w[0] = ctx->wg[l];
-    gu.w[1] = ctx->wu[l];
-    gu.seg_rows[0] = gu.seg_rows[1] = c.intermediate;
-    gu.tag = TAG_GATEUP;
-    gu.epi.kind = EPI_SWIGLU;
-    gu.epi.out_type = OUT_BF16X2;
-    gu.epi.out_plane = (size_t)R * c.intermediate;
-    gu.epi.out[0] = ctx->act;
-    gu.epi.ld_out[0] = c.intermediate;
-    set_deferred_norm(ctx, gu.epi, ctx->sumsq[0], R);
-    DFL_CHECK(run_gemm(ctx, gu, st));
+    for (int l = 0; l < c.n_layers; ++l) {
+      GemmSpec qkv;
+      qkv.x = ctx->h;
+      qkv.x_split = ctx->bf16;
+      qkv.ldx = H;
+      qkv.M = R;
+      qkv.K = H;
+      qkv.n_seg = 3;
+      qkv.w[0] = ctx->wq[l];
+      qkv.w[1] = ctx->wk[l];
+      qkv.w[2] = ctx->wv[l];
+      qkv.seg_rows[0] = QD;
+      qkv.seg_rows[1] = KVD;
+      qkv.seg_rows[2] = KVD;
+      qkv.tag = TAG_QKV;
+      qkv.epi.kind = EPI_QKV;
+      qkv.epi.out_type = OUT_F16;   // the attention kernel runs in fp16
+      qkv.epi.out[0] = ctx->q;
+      qkv.epi.out[1] = ctx->kb;
+      qkv.epi.out[2] = ctx->vb;
+      qkv.epi.ld_out[0] = QD;
+      qkv.epi.ld_out[1] = KVD;
+      qkv.epi.ld_out[2] = KVD;
+      qkv.epi.rope_mask = 3u;
+      qkv.epi.head_dim = c.head_dim;
+      qkv.epi.inv_freq = ctx->inv_freq;
+      qkv.epi.rows_per_req = B;
+      qkv.epi.pos_base = d_ctx_len;
+      if (l > 0) set_deferred_norm(ctx, qkv.epi, ctx->sumsq[1], R);   // rows carry the previous layer's norm
+      DFL_CHECK(run_gemm(ctx, qkv, st));
 
-    GemmSpec dn;
-    dn.x = ctx->act;
-    dn.x_split = ctx->bf16;
-    dn.ldx = c.intermediate;
-    dn.M = R;
-    dn.K = c.intermediate;
-    dn.n_seg = 1;
-    dn.w[0] = ctx->wd[l];
-    dn.seg_rows[0] = H;
-    dn.tag = TAG_DOWN;
-    dn.epi.kind = EPI_RESID;
-    dn.epi.x = ctx->x;
-    dn.epi.ldx = H;
-    // the next layer's attention norm (or the final norm) is deferred the same way
-    const bool last = l + 1 == c.n_layers;
-    dn.epi.gamma_next = last ? ctx->final_norm : ctx->attn_norm[l + 1];
-    dn.epi.out_type = OUT_BF16X2;
-    dn.epi.out_plane = (size_t)R * H;
-    dn.epi.xg = ctx->h;
-    dn.epi.sumsq = ctx->sumsq[1];
-    dn.epi.ld_part = R;
-    DFL_CHECK(run_gemm(ctx, dn, st));
+      AttnParams ap{};
+      ap.q = ctx->q;
+      ap.kblk = ctx->kb;
+      ap.vblk = ctx->vb;
+      ap.kc = k_cache[l];
+      ap.vc = v_cache[l];
+      ap.ctx_len = d_ctx_len;
+      ap.page_table = d_page_table;
+      ap.max_pages = max_pages;
+      ap.num_pages = num_pages;
+      ap.page_size = c.page_size;
+      ap.bs = bs;
+      ap.B = B;
+      ap.n_q = c.n_q_heads;
+      ap.n_kv = c.n_kv_heads;
+      ap.d = c.head_dim;
+      ap.g = g;
+      ap.kps = kps;
+      ap.n_splits = n_splits;
+      ap.ks = attn_ks;
+      ap.global_merge = attn_gmerge ? 1 : 0;
+      ap.max_ctx = max_ctx;
+      ap.scale = (float)(1.0 / std::sqrt((double)c.head_dim));
+      ap.part_o = ctx->att_o;
+      ap.part_m = ctx->att_m;
+      ap.part_l = ctx->att_l;
+      ap.status = ctx->status;
+      ap.out_plane = (size_t)R * QD;
+      ap.cache_f16 = ctx->cache_f16 ? 1 : 0;
+      {
+        // context K/V of every request (upper bound max_ctx), block q/k/v, output
+        const double kvb = (double)bs * max_ctx * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;
+        const double fl = 4.0 * bs * B * (double)(max_ctx + B) * QD;
+        ProfScope prof(ctx, PK_ATTN, st, kvb, fl);
+        DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, hb, hb, st, ctx->use_pdl), "attention launch"));
+      }
 
-    if (d_hidden_out) {
-      ProfScope prof(ctx, PK_COPY, st, (double)layer_stride * 8, 0);
-      if (cudaMemcpyAsync(d_hidden_out + l * layer_stride, ctx->x, layer_stride * 4, cudaMemcpyDeviceToDevice,
-                          st) != cudaSuccess)
-        return DFLASH_ERR_CUDA;
-      if (last) {
-        // the final normed rows, for parity checks only (the LM head uses the deferred form)
-        ProfScope prof2(ctx, PK_RMSNORM, st, norm_bytes, 0);
-        DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, nullptr, hb,
-                                             d_hidden_out + (size_t)c.n_layers * layer_stride, st, ctx->use_pdl),
-                              "rmsnorm launch"));
+      GemmSpec o;
+      o.x = ctx->ao;
+      o.x_split = ctx->bf16;
+      o.ldx = QD;
+      o.M = R;
+      o.K = QD;
+      o.n_seg = 1;
+      o.w[0] = ctx->wo[l];
+      o.seg_rows[0] = H;
+      o.tag = TAG_O;
+      o.epi.kind = EPI_RESID;
+      o.epi.x = ctx->x;
+      o.epi.ldx = H;
+      // the MLP norm is deferred: x ⊙ gain now, the row scales in the gate/up epilogue
+      o.epi.gamma_next = ctx->mlp_norm[l];
+      o.epi.out_type = OUT_BF16X2;
+      o.epi.out_plane = (size_t)R * H;
+      o.epi.xg = ctx->h;
+      o.epi.sumsq = ctx->sumsq[0];
+      o.epi.ld_part = R;
+      DFL_CHECK(run_gemm(ctx, o, st));
+
+      GemmSpec gu;
+      gu.x = ctx->h;
+      gu.x_split = ctx->bf16;
+      gu.ldx = H;
+      gu.M = R;
+      gu.K = H;
+      gu.n_seg = 2;
+      gu.paired = true;
+      gu.w[0] = ctx->wg[l];
+      gu.w[1] = ctx->wu[l];
+      gu.seg_rows[0] = gu.seg_rows[1] = c.intermediate;
+      gu.tag = TAG_GATEUP;
+      gu.epi.kind = EPI_SWIGLU;
+      gu.epi.out_type = OUT_BF16X2;
+      gu.epi.out_plane = (size_t)R * c.intermediate;
+      gu.epi.out[0] = ctx->act;
+      gu.epi.ld_out[0] = c.intermediate;
+      set_deferred_norm(ctx, gu.epi, ctx->sumsq[0], R);
+      DFL_CHECK(run_gemm(ctx, gu, st));
+
+      GemmSpec dn;
+      dn.x = ctx->act;
+      dn.x_split = ctx->bf16;
+      dn.ldx = c.intermediate;
+      dn.M = R;
+      dn.K = c.intermediate;
+      dn.n_seg = 1;
+      dn.w[0] = ctx->wd[l];
+      dn.seg_rows[0] = H;
+      dn.tag = TAG_DOWN;
+      dn.epi.kind = EPI_RESID;
+      dn.epi.x = ctx->x;
+      dn.epi.ldx = H;
+      // the next layer's attention norm (or the final norm) is deferred the same way
+      const bool last = l + 1 == c.n_layers;
+      dn.epi.gamma_next = last ? ctx->final_norm : ctx->attn_norm[l + 1];
+      dn.epi.out_type = OUT_BF16X2;
+      dn.epi.out_plane = (size_t)R * H;
+      dn.epi.xg = ctx->h;
+      dn.epi.sumsq = ctx->sumsq[1];
+      dn.epi.ld_part = R;
+      DFL_CHECK(run_gemm(ctx, dn, st));
+
+      if (d_hidden_out) {
+        ProfScope prof(ctx, PK_COPY, st, (double)layer_stride * 8, 0);
+        if (cudaMemcpyAsync(d_hidden_out + l * layer_stride, ctx->x, layer_stride * 4, cudaMemcpyDeviceToDevice,
+                            st) != cudaSuccess)
+          return DFLASH_ERR_CUDA;
+        if (last) {
+          // the final normed rows, for parity checks only (the LM head uses the deferred form)
+          ProfScope prof2(ctx, PK_RMSNORM, st, norm_bytes, 0);
+          DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, nullptr, hb,
+                                               d_hidden_out + (size_t)c.n_layers * layer_stride, st, ctx->use_pdl),
+                                "rmsnorm launch"));
+        }
       }
     }
-  }
-  if (c.n_layers == 0 && d_hidden_out)
-    DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, ctx->h, hb, d_hidden_out, st,
-                                         ctx->use_pdl),
-                          "rmsnorm launch"));
+    if (c.n_layers == 0 && d_hidden_out)
+      DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, ctx->h, hb, d_hidden_out, st,
+                                           ctx->use_pdl),
+                            "rmsnorm launch"));
 
-  GemmSpec lm;
-  lm.x = ctx->h;
-  // The LM head only feeds an argmax: above 32 rows it reads the hi plane alone,
-  // which halves its MMA work and activation tiles (from 64 rows on, the split
-  // makes it tensor- or shared-memory-bound). The hi plane's rounding (2^-9
-  // relative) moves a logit by ~2e-3 (std) at these scales, inside the 1e-2
-  // top-2 gap the draft tokens are held to; up to 32 rows the lo plane is free.
-  lm.x_split = ctx->bf16 && R <= 32;
-  lm.ldx = H;
-  lm.M = R;
-  lm.K = H;
-  lm.n_seg = 1;
-  lm.w[0] = ctx->lm_head;
-  lm.seg_rows[0] = c.vocab;
-  lm.tag = TAG_LM;
-  lm.epi.kind = EPI_ARGMAX;
-  lm.epi.keys = ctx->keys;
-  if (c.n_layers > 0) set_deferred_norm(ctx, lm.epi, ctx->sumsq[1], R);
-  DFL_CHECK(run_gemm(ctx, lm, st));
-  {
-    ProfScope prof(ctx, PK_ARGMAX, st, (double)R * 8 * 2 + (double)bs * (B - 1) * 4, 0);
-    DFL_CHECK(cuda_status(launch_argmax_finalize(ctx->keys, bs, B, d_draft, st, ctx->use_pdl),
-                          "argmax_finalize launch"));
+    GemmSpec lm;
+    lm.x = ctx->h;
+    // The LM head only feeds an argmax: above 32 rows it reads the hi plane alone,
+    // which halves its MMA work and activation tiles (from 64 rows on, the split
+    // makes it tensor- or shared-memory-bound). The hi plane's rounding (2^-9
+    // relative) moves a logit by ~2e-3 (std) at these scales, inside the 1e-2
+    // top-2 gap the draft tokens are held to; up to 32 rows the lo plane is free.
+    lm.x_split = ctx->bf16 && R <= 32;
+    lm.ldx = H;
+    lm.M = R;
+    lm.K = H;
+    lm.n_seg = 1;
+    lm.w[0] = ctx->lm_head;
+    lm.seg_rows[0] = c.vocab;
+    lm.tag = TAG_LM;
+    lm.epi.kind = EPI_ARGMAX;
+    lm.epi.keys = ctx->keys;
+    if (c.n_layers > 0) set_deferred_norm(ctx, lm.epi, ctx->sumsq[1], R);
+    DFL_CHECK(run_gemm(ctx, lm, st));
+    {
+      ProfScope prof(ctx, PK_ARGMAX, st, (double)R * 8 * 2 + (double)bs * (B - 1) * 4, 0);
+      DFL_CHECK(cuda_status(launch_argmax_finalize(ctx->keys, bs, B, d_draft, st, ctx->use_pdl),
+                            "argmax_finalize launch"));
+    }
+    return DFLASH_OK;
+  } catch (...) {   // no C++ exception crosses the C ABI
+    return DFLASH_ERR_OOM;
   }
-  return DFLASH_OK;
 }
