@@ -38,8 +38,11 @@
  *     the previous cycle's result.
  *   - Weights and features are bf16 or fp32 (dflash_config.dtype); the KV
  *     cache is the same type or, for a bf16 drafter, fp16
- *     (dflash_config.cache_dtype); RMSNorm gains are always fp32. Accumulation is fp32; the draft argmax is taken on
- *     fp32 logits, which are never written to memory.
+ *     (dflash_config.cache_dtype); RMSNorm gains are always fp32.
+ *     Accumulation is fp32; the draft argmax is taken on fp32 logits, which
+ *     are never written to memory.
+ *   - No C++ exception crosses this interface: a failed host allocation is
+ *     returned as DFLASH_ERR_OOM.
  */
 #ifndef DFLASH_H
 #define DFLASH_H
@@ -55,7 +58,7 @@ typedef enum {
   DFLASH_OK = 0,
   DFLASH_ERR_ARG = 1,          /* invalid argument (host-side check) */
   DFLASH_ERR_CUDA = 2,         /* a CUDA runtime / driver call failed */
-  DFLASH_ERR_OOM = 3,          /* workspace allocation failed (dflash_create only) */
+  DFLASH_ERR_OOM = 3,          /* device workspace (dflash_create) or host allocation failed */
   DFLASH_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up */
   DFLASH_ERR_DEVICE = 5,       /* a kernel met an out-of-range id, page or position */
   DFLASH_ERR_UNSUPPORTED = 6   /* a shape this build has no kernel for */
