@@ -62,6 +62,7 @@ struct dflash_ctx {
   int force_splits = 0;   // DFLASH_SPLITS: fixed K-split count (experiments)
   int force_stages = 0;   // DFLASH_STAGES: fixed ring depth (experiments)
   int split_slots = 2;    // CTAs per SM the K-split plan fills (DFLASH_SPLIT_SLOTS, experiments)
+  unsigned test_stall_ns = 0;   // DFLASH_TEST_STALL_NS: failure-injection hook of the tensor-core GEMM
   int num_sms = 148;
   const void* fc = nullptr;
   const void* embed = nullptr;
@@ -268,6 +269,7 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
     std::fprintf(stderr, "dflash gemm tag=%d M=%d K=%d tiles=%d m_tile=%d stages=%d splits=%d\n", g.tag, g.M, g.K,
                  n_tiles, p.m_tile, p.stages, p.splits);
   p.use_pdl = ctx->use_pdl ? 1 : 0;
+  p.test_stall_ns = ctx->test_stall_ns;
   const int box_w = g.paired ? kTileN / 2 : kTileN;
   const int nmaps = g.paired ? 2 : g.n_seg;
   for (int s = 0; s < nmaps; ++s)
@@ -351,6 +353,14 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     if (ctx->force_stages > 8) ctx->force_stages = 8;
     env = std::getenv("DFLASH_PDL");
     ctx->use_pdl = !(env && env[0] == '0');
+    // Failure injection (tests only): every tensor-core GEMM epilogue gives up on a
+    // barrier nothing arrives at after this many ns (capped at 100 ms), so the
+    // call completes with DFLASH_ERR_TIMEOUT and no copy or MMA in flight.
+    env = std::getenv("DFLASH_TEST_STALL_NS");
+    if (env) {
+      const long long v = std::atoll(env);
+      ctx->test_stall_ns = v <= 0 ? 0u : (unsigned)std::min(v, 100000000LL);
+    }
     int dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev);
@@ -836,8 +846,14 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     DFL_CHECK(run_gemm(ctx, lm, st));
     {
       ProfScope prof(ctx, PK_ARGMAX, st, (double)R * 8 * 2 + (double)bs * (B - 1) * 4, 0);
-      DFL_CHECK(cuda_status(launch_argmax_finalize(ctx->keys, bs, B, d_draft, st, ctx->use_pdl),
-                            "argmax_finalize launch"));
+      const dflash_status fs = cuda_status(launch_argmax_finalize(ctx->keys, bs, B, d_draft, st, ctx->use_pdl),
+                                           "argmax_finalize launch");
+      if (fs != DFLASH_OK) {
+        // the LM head has folded its maxima into the keys: clear them, or the next
+        // draft would start from this call's keys
+        cudaMemsetAsync(ctx->keys, 0, (size_t)R * sizeof(unsigned long long), st);
+        return fs;
+      }
     }
     return DFLASH_OK;
   } catch (...) {   // no C++ exception crosses the C ABI

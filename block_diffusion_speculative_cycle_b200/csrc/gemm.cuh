@@ -288,6 +288,11 @@ struct alignas(64) GemmTcParams {
   int n_tiles;
   int stages;
   int use_pdl;
+  // Failure-injection hook, 0 in normal use: when set, every epilogue thread,
+  // once the accumulator is final, also waits on a barrier nothing ever arrives
+  // at, bounded by this many ns, so the bounded-wait give-up path runs (ST_TIMEOUT
+  // flagged, epilogue skipped, TMEM freed) with no copy or MMA in flight.
+  unsigned int test_stall_ns;
 };
 
 cudaError_t launch_gemm_simt(const GemmSimtParams& p, int n_tiles, cudaStream_t st, bool pdl);

@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
   __shared__ uint64_t empty_bar[kMaxStages];
   __shared__ uint64_t acc_bar;
   __shared__ uint64_t recv_bar;
+  __shared__ uint64_t stall_bar;   // failure-injection hook only: never arrived at
   __shared__ uint32_t tmem_slot;
   __shared__ int s_flag;
   __shared__ float epi_scratch[kEpiScratch];
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
     }
     mbar_init(&acc_bar, 1);
     mbar_init(&recv_bar, 1);
+    mbar_init(&stall_bar, 1);
     s_flag = 0;
     fence_mbar_init();
     if (p.splits > 1) mbar_arrive_expect_tx(&recv_bar, (uint32_t)(p.splits * (own_hi - own_lo) * kTileN * 4));
@@ -185,7 +187,9 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
     grid_dep_wait();   // epilogue reads / writes data shared with the previous kernel
     // the row scales depend only on earlier kernels: compute them while the MMAs run
     epilogue_row_scales(p.epi, row0, rows_here, row_scale, t);
-    const bool got = nkb > 0 ? mbar_wait(&acc_bar, 0, status) : true;
+    bool got = nkb > 0 ? mbar_wait(&acc_bar, 0, status) : true;
+    // failure-injection hook: a wait that can only run out (nothing is in flight now)
+    if (p.test_stall_ns && got) got = mbar_wait(&stall_bar, 0, status, p.test_stall_ns);
     // one decision for all 128 threads (the MMA lane may set s_flag at any time)
     bool ok = !named_bar_or(1, 128, !got || s_flag != 0) && nkb > 0;
     tc_fence_after();

@@ -10,7 +10,7 @@ Sources (page title, section):
        feature extraction, KV injection into the drafter KV cache, parallel block
        prediction), §2.3 (embedding and LM head shared with the target, frozen)
 
-Readings where the pages are silent (each listed with its reason in the design doc):
+Readings where the pages are silent (each the plainest one the rest of the pages support):
   * the projection is one bias-free linear map, no norm after it;
   * each layer injects with its own Wk/Wv, without that layer's input RMSNorm;
     K gets RoPE at the context token's absolute position;

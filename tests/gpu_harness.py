@@ -51,15 +51,20 @@ class PagedCache:
         return self.table.shape[1]
 
 
+def slots_of(pos: np.ndarray, page_size: int) -> np.ndarray:
+    return (pos % page_size).astype(np.int64)
+
+
 def gather_cpu_cache(cfg, pools_cpu, table_cpu: torch.Tensor, r: int, P: int, page_size: int):
     """Oracle view of request r's first P positions from CPU page pools (synth input)."""
     ks, vs = [], []
     pos = np.arange(P)
-    pages = table_cpu[r].numpy()[pos // page_size]
-    slots = pos % page_size
+    pages = torch.as_tensor(table_cpu[r].numpy()[pos // page_size].astype(np.int64))
+    slots = torch.as_tensor(slots_of(pos, page_size))
     for lay in pools_cpu:
-        k = O.f64(lay["k"])[pages, :, slots, :]   # [P, n_kv, d]
-        v = O.f64(lay["v"])[pages, :, slots, :]
+        # gather this request's rows first, then widen only those
+        k = O.f64(lay["k"][pages, :, slots, :])   # [P, n_kv, d]
+        v = O.f64(lay["v"][pages, :, slots, :])
         ks.append(k)
         vs.append(v)
     return O.Cache.from_arrays(cfg, ks, vs)

@@ -16,7 +16,7 @@ from tests.gpu_harness import PagedCache, make_drafter
 
 pytestmark = pytest.mark.gpu
 
-ERR_ARG, ERR_DEVICE = 1, 5
+ERR_ARG, ERR_TIMEOUT, ERR_DEVICE = 1, 4, 5
 
 SMALL_BF16 = synth.DrafterConfig(name="small-bf16", hidden=512, n_layers=2, n_q_heads=4, n_kv_heads=2,
                                  head_dim=128, intermediate=1024, vocab=2048, n_feat_layers=3,
@@ -101,3 +101,34 @@ def test_host_argument_errors_launch_nothing():
     assert e.value.status == ERR_ARG
     drafter.check()
     drafter.close()
+
+
+def test_a_device_wait_that_runs_out_reports_timeout_and_a_fresh_context_works(monkeypatch):
+    """Failure injection without a fault: with DFLASH_TEST_STALL_NS set when the
+    context is created, every tensor-core GEMM epilogue also waits on a barrier
+    that nothing arrives at, bounded by 1 ms. Injection and the draft pass must
+    come back, each report DFLASH_ERR_TIMEOUT once, and a context created
+    afterwards without the hook must match the oracle again."""
+    from tests.test_gpu_draft import run_case
+    cfg, ctx_len, B = SMALL_BF16, 128, 4
+    monkeypatch.setenv("DFLASH_TEST_STALL_NS", "1000000")
+    w = synth.make_drafter_weights(cfg, seed=0)
+    ctx = torch.tensor([ctx_len], dtype=torch.int32)
+    table, num_pages = synth.make_page_table(ctx, 64, extra_tokens=B, seed=1)
+    drafter, _ = make_drafter(cfg, w, max_block=B, max_batch=1, max_inject_rows=ctx_len, page_size=64)
+    monkeypatch.delenv("DFLASH_TEST_STALL_NS")
+    cache = PagedCache(cfg, table, num_pages, 64)
+    feats = synth.make_features(cfg, ctx_len, seed=2).reshape(1, ctx_len, cfg.feat_dim).cuda()
+    n_new = torch.tensor([ctx_len], dtype=torch.int32, device="cuda")
+    start = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for step in ("inject", "draft"):
+        if step == "inject":
+            drafter.inject(feats, 1, ctx_len, n_new, start, cache.k, cache.v, cache.table, num_pages)
+        else:
+            draft(drafter, cache, num_pages, torch.tensor([3], dtype=torch.int32), ctx, B)
+        with pytest.raises(DFlashError) as e:
+            drafter.check()
+        assert e.value.status == ERR_TIMEOUT, step
+        drafter.check()   # reported once
+    drafter.close()
+    run_case(cfg, [200], 16, seed=21)
