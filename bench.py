@@ -225,13 +225,16 @@ class Cycle:
 
 
 def algorithmic_cycle_bytes(c) -> float:
-    """Weights read once, the context K/V each request attends to, features,
-    logits; activations are negligible at these sizes."""
+    """Every weight the cycle reads, once per use: the drafter layers' weights,
+    the LM head and the fusion projection, plus every layer's Wk and Wv a second
+    time for the injection; the context K/V each request attends to, the
+    features and the block logits. Activations are negligible at these sizes."""
     cfg = c.cfg
     es = 2 if cfg.dtype == "bf16" else 4
     H, I, L = cfg.hidden, cfg.intermediate, cfg.n_layers
     per_layer = (2 * cfg.q_dim * H + 2 * cfg.kv_dim * H + 3 * I * H) * es
-    weights = L * per_layer + cfg.vocab * H * es + H * cfg.feat_dim * es
+    inject_kv = L * 2 * cfg.kv_dim * H * es
+    weights = L * per_layer + cfg.vocab * H * es + H * cfg.feat_dim * es + inject_kv
     kv = float(c.ctx_lens.sum()) * L * 2 * cfg.kv_dim * es
     feats = c.bs * c.B * cfg.feat_dim * es
     logits = c.bs * c.B * cfg.vocab * 2
@@ -259,6 +262,17 @@ class HostCycle:
                                                              seed=w.seed + 6, dtype=torch.bfloat16)
         self.n_new_cpu = torch.clamp(self.planted + 1, max=B).to(torch.int32)
         self.start_cpu = (self.ctx_lens - self.n_new_cpu).clamp(min=0).to(torch.int32)
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown CPU"
 
 
 def oracle_cycle_estimate(c, budget_s: float):
@@ -309,9 +323,9 @@ def oracle_cycle_estimate(c, budget_s: float):
             cores = max(p.get("num_threads", 1) for p in info)
     except Exception:
         pass
-    sample = (f"1 of {c.bs} requests; inject {int(c.n_new_cpu[0])} rows + 1 of {cfg.n_layers} layers "
-              f"(context {P}) + final norm and LM head on 1/{n_slices} of the vocab + verify; "
-              f"{len(times['layer'])} repeats, median, extrapolated to the full batch cycle")
+    sample = (f"float64 NumPy oracle on {cpu_model()}: 1 of {c.bs} requests; inject {int(c.n_new_cpu[0])} rows "
+              f"+ 1 of {cfg.n_layers} layers (context {P}) + final norm and LM head on 1/{n_slices} of the vocab "
+              f"+ verify; {len(times['layer'])} repeats, median, extrapolated to the full batch cycle")
     return 1.0 / cycle_s, cores, sample
 
 
@@ -321,13 +335,10 @@ def run_reference(args, world, rank):
     """The oracle on the host cores, same workload / metric / unit as our arm."""
     if rank != 0:
         return
-    import torch
     from block_diffusion_speculative_cycle_b200 import synth
     w = synth.WORKLOADS[args.workload]
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-
-    # reuse Cycle's input construction on the GPU if present (for the planted logits), else CPU-only inputs
-    c = Cycle(w, dev, args.kv_cache_dtype) if dev == "cuda" else HostCycle(w, args.kv_cache_dtype)
+    # inputs built on the host only: this arm never loads the CUDA library
+    c = HostCycle(w, args.kv_cache_dtype)
     steps = max(1, args.steps)
     budget_per_step = max(2.0, 150.0 / (steps + args.warmup))
     vals = []
@@ -433,6 +444,33 @@ def run_ours(args, world, rank, local):
     pk = peaks()
     dom = max(kinds.values(), key=lambda e: e["total_ms"])
     avg_s = dom["total_ms"] / dom["launches"] / 1000.0
+    timing = "eager, an event pair around every launch (no overlap between launches)"
+    if dom["name"] == "gemm_tc":
+        # Inside the cycle the GEMMs overlap each other's ramp and tail (programmatic
+        # dependent launch), which event pairs around single launches remove: time a
+        # CUDA graph of exactly the cycle's GEMM launches instead, K replays.
+        from block_diffusion_speculative_cycle_b200 import dflash_profile_gemm_chain
+        g3 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g3, stream=stream):
+            dflash_profile_gemm_chain(c.drafter.handle, c.feats, c.bs, c.B, c.n_new, c.start, c.kc, c.vc, c.table,
+                                      c.num_pages, c.ctx, c.B)
+        for _ in range(3):
+            g3.replay()
+        torch.cuda.synchronize()
+        ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(3, min(args.steps, 100))
+        ga.record()
+        for _ in range(reps):
+            g3.replay()
+        gb.record()
+        torch.cuda.synchronize()
+        c.drafter.check()
+        chain_s = ga.elapsed_time(gb) / 1000.0 / reps
+        per_cycle = dom["launches"] / args.profile_steps
+        avg_s = chain_s / per_cycle
+        timing = (f"in-cycle: a CUDA graph of the cycle's {per_cycle:.0f} GEMM launches (programmatic dependent "
+                  f"launch on), {reps} replays, {1e6 * chain_s:.1f} us per cycle")
+        del g3
     bytes_per_launch = dom["bytes"] / dom["launches"]
     flops_per_launch = dom["flops"] / dom["launches"]
     intensity = flops_per_launch / max(bytes_per_launch, 1.0)
@@ -446,6 +484,9 @@ def run_ours(args, world, rank, local):
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
                 "frac": achieved / pk["hbm"], "peak_source": f"{pk['src']} hbm copy"}
     roof["kernel"] = dom["name"]
+    roof["us_per_launch"] = 1e6 * avg_s
+    roof["bytes_per_launch"] = bytes_per_launch
+    roof["timing"] = timing
     roof["traffic"] = stored_traffic(dom["name"], w.name)
     cycle_bytes = algorithmic_cycle_bytes(c)
     per_gpu_cycle_s = (ms_max / 1000.0) / args.steps

@@ -7,6 +7,7 @@ is no CPU fallback).
 """
 from ._binding import (  # noqa: F401
     DFLASH_BF16, DFLASH_F16, DFLASH_F32, DFlashError, Drafter, dflash_create, dflash_destroy, dflash_draft_block,
-    dflash_get_error, dflash_inject_ctx, dflash_profile_enable, dflash_profile_read, dflash_status_string, dflash_verify, dflash_verify_workspace_size,
+    dflash_get_error, dflash_inject_ctx, dflash_profile_enable, dflash_profile_gemm_chain, dflash_profile_read,
+    dflash_status_string, dflash_verify, dflash_verify_workspace_size,
     exported_symbols, load_library, verify,
 )

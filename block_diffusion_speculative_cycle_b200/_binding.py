@@ -23,7 +23,7 @@ _STATUS = {0: "DFLASH_OK", 1: "DFLASH_ERR_ARG", 2: "DFLASH_ERR_CUDA", 3: "DFLASH
 
 EXPORTS = ["dflash_create", "dflash_destroy", "dflash_inject_ctx", "dflash_draft_block",
            "dflash_verify_workspace_size", "dflash_verify", "dflash_verify_noalloc", "dflash_profile_enable", "dflash_profile_read",
-           "dflash_get_error", "dflash_status_string"]
+           "dflash_profile_gemm_chain", "dflash_get_error", "dflash_status_string"]
 
 
 class DFlashError(RuntimeError):
@@ -87,6 +87,8 @@ def load_library(path: Optional[str] = None):
     lib.dflash_profile_enable.restype = c_int
     lib.dflash_profile_read.argtypes = [_P, ctypes.POINTER(dflash_profile_entry), c_int]
     lib.dflash_profile_read.restype = c_int
+    lib.dflash_profile_gemm_chain.argtypes = [_P, _P, c_int, c_int, _P, _P, _PP, _PP, _P, c_int, c_int, _P, c_int, _P]
+    lib.dflash_profile_gemm_chain.restype = c_int
     lib.dflash_get_error.argtypes = [_P, _P]
     lib.dflash_get_error.restype = c_int
     lib.dflash_status_string.argtypes = [c_int]
@@ -188,6 +190,15 @@ def dflash_profile_read(handle) -> List[dict]:
         raise DFlashError(-n, "dflash_profile_read")
     return [{"name": arr[i].name.decode(), "launches": arr[i].launches, "total_ms": arr[i].total_ms,
              "bytes": arr[i].bytes, "flops": arr[i].flops} for i in range(n)]
+
+
+def dflash_profile_gemm_chain(handle, feats, bs, max_new, n_new, start_pos, k_cache, v_cache, page_table,
+                              num_pages, ctx_len, B, stream=None) -> None:
+    lib = load_library()
+    _check(lib.dflash_profile_gemm_chain(handle, _ptr(feats), bs, max_new, _ptr(n_new), _ptr(start_pos),
+                                         _ptr_array(k_cache), _ptr_array(v_cache), _ptr(page_table),
+                                         page_table.shape[1], num_pages, _ptr(ctx_len), B, _stream(stream)),
+           "dflash_profile_gemm_chain")
 
 
 def dflash_get_error(handle, stream=None) -> int:

@@ -63,6 +63,9 @@ struct dflash_ctx {
   int force_stages = 0;   // DFLASH_STAGES: fixed ring depth (experiments)
   int split_slots = 2;    // CTAs per SM the K-split plan fills (DFLASH_SPLIT_SLOTS, experiments)
   unsigned test_stall_ns = 0;   // DFLASH_TEST_STALL_NS: failure-injection hook of the tensor-core GEMM
+  bool attn_mma = false;        // DFLASH_ATTN=mma: the mma.sync attention kernel even where tcgen05 applies
+  int attn_stages = 4;          // K/V ring depth of the tcgen05 attention (DFLASH_ATTN_STAGES, experiments)
+  std::map<std::tuple<int, int, int, int>, int> attn_cluster_cap;   // resident clusters per (d, stages, n, rows)
   int num_sms = 148;
   const void* fc = nullptr;
   const void* embed = nullptr;
@@ -93,6 +96,7 @@ struct dflash_ctx {
   bool prof = false;
   std::vector<ProfRec> recs;
   std::map<std::tuple<const void*, long long, long long, long long, int>, CUtensorMap> maps;
+  std::map<std::vector<long long>, CUtensorMap> maps_nd;   // fp16 tensor maps of the attention kernel
 };
 
 namespace {
@@ -149,6 +153,40 @@ bool get_map(dflash_ctx* ctx, const void* ptr, long long rows, long long K, long
   if (r != CUDA_SUCCESS) return false;
   if (ctx->maps.size() > 4096) ctx->maps.clear();
   ctx->maps[key] = m;
+  *out = m;
+  return true;
+}
+
+// fp16 tensor map (128-byte swizzle, zero fill out of bounds), rank 2 or 3;
+// dims / box in elements (innermost first), strides in bytes of dims 1.. .
+bool get_map_f16(dflash_ctx* ctx, const void* ptr, int rank, const long long* dims, const long long* strides,
+                 const int* box, CUtensorMap* out) {
+  std::vector<long long> key = {(long long)(uintptr_t)ptr, rank};
+  for (int i = 0; i < rank; ++i) key.push_back(dims[i]);
+  for (int i = 0; i + 1 < rank; ++i) key.push_back(strides[i]);
+  for (int i = 0; i < rank; ++i) key.push_back(box[i]);
+  auto it = ctx->maps_nd.find(key);
+  if (it != ctx->maps_nd.end()) {
+    *out = it->second;
+    return true;
+  }
+  cuuint64_t d[3], st[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = (cuuint64_t)dims[i];
+    bx[i] = (cuuint32_t)box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = (cuuint64_t)strides[i];
+  CUtensorMap m;
+  CUresult r = ctx->encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), d, st, bx,
+                           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::fprintf(stderr, "dflash: tensor map encode failed (%d)\n", (int)r);
+    return false;
+  }
+  if (ctx->maps_nd.size() > 4096) ctx->maps_nd.clear();
+  ctx->maps_nd[key] = m;
   *out = m;
   return true;
 }
@@ -288,6 +326,144 @@ void set_deferred_norm(dflash_ctx* ctx, EpiParams& e, const float* part, int row
   e.norm_eps = ctx->cfg.rms_eps;
 }
 
+// ---------------------------------------------------------------- the draft pass's GEMMs
+// (R = bs * B activation rows; one builder per call site, shared by
+// dflash_draft_block and the GEMM-chain instrumentation call)
+
+// RMSNorm -> q, k, v of the block rows, RoPE on q and k at positions ctx_len + i.
+GemmSpec spec_qkv(dflash_ctx* ctx, int l, int R, int B, const int* d_ctx_len) {
+  const dflash_config& c = ctx->cfg;
+  const int QD = q_dim(c), KVD = kv_dim(c);
+  GemmSpec qkv;
+  qkv.x = ctx->h;
+  qkv.x_split = ctx->bf16;
+  qkv.ldx = c.hidden;
+  qkv.M = R;
+  qkv.K = c.hidden;
+  qkv.n_seg = 3;
+  qkv.w[0] = ctx->wq[l];
+  qkv.w[1] = ctx->wk[l];
+  qkv.w[2] = ctx->wv[l];
+  qkv.seg_rows[0] = QD;
+  qkv.seg_rows[1] = KVD;
+  qkv.seg_rows[2] = KVD;
+  qkv.tag = TAG_QKV;
+  qkv.epi.kind = EPI_QKV;
+  qkv.epi.out_type = OUT_F16;   // the attention kernels run in fp16
+  qkv.epi.out[0] = ctx->q;
+  qkv.epi.out[1] = ctx->kb;
+  qkv.epi.out[2] = ctx->vb;
+  qkv.epi.ld_out[0] = QD;
+  qkv.epi.ld_out[1] = KVD;
+  qkv.epi.ld_out[2] = KVD;
+  qkv.epi.rope_mask = 3u;
+  qkv.epi.head_dim = c.head_dim;
+  qkv.epi.inv_freq = ctx->inv_freq;
+  qkv.epi.rows_per_req = B;
+  qkv.epi.pos_base = d_ctx_len;
+  if (l > 0) set_deferred_norm(ctx, qkv.epi, ctx->sumsq[1], R);   // rows carry the previous layer's norm
+  return qkv;
+}
+
+// x += o · Woᵀ; the MLP norm is deferred: x ⊙ gain now, the row scales in the gate/up epilogue.
+GemmSpec spec_o(dflash_ctx* ctx, int l, int R) {
+  const dflash_config& c = ctx->cfg;
+  GemmSpec o;
+  o.x = ctx->ao;
+  o.x_split = ctx->bf16;
+  o.ldx = q_dim(c);
+  o.M = R;
+  o.K = q_dim(c);
+  o.n_seg = 1;
+  o.w[0] = ctx->wo[l];
+  o.seg_rows[0] = c.hidden;
+  o.tag = TAG_O;
+  o.epi.kind = EPI_RESID;
+  o.epi.x = ctx->x;
+  o.epi.ldx = c.hidden;
+  o.epi.gamma_next = ctx->mlp_norm[l];
+  o.epi.out_type = OUT_BF16X2;
+  o.epi.out_plane = (size_t)R * c.hidden;
+  o.epi.xg = ctx->h;
+  o.epi.sumsq = ctx->sumsq[0];
+  o.epi.ld_part = R;
+  return o;
+}
+
+// act = silu(h · Wgᵀ) ⊙ (h · Wuᵀ), paired gate / up tiles.
+GemmSpec spec_gateup(dflash_ctx* ctx, int l, int R) {
+  const dflash_config& c = ctx->cfg;
+  GemmSpec gu;
+  gu.x = ctx->h;
+  gu.x_split = ctx->bf16;
+  gu.ldx = c.hidden;
+  gu.M = R;
+  gu.K = c.hidden;
+  gu.n_seg = 2;
+  gu.paired = true;
+  gu.w[0] = ctx->wg[l];
+  gu.w[1] = ctx->wu[l];
+  gu.seg_rows[0] = gu.seg_rows[1] = c.intermediate;
+  gu.tag = TAG_GATEUP;
+  gu.epi.kind = EPI_SWIGLU;
+  gu.epi.out_type = OUT_BF16X2;
+  gu.epi.out_plane = (size_t)R * c.intermediate;
+  gu.epi.out[0] = ctx->act;
+  gu.epi.ld_out[0] = c.intermediate;
+  set_deferred_norm(ctx, gu.epi, ctx->sumsq[0], R);
+  return gu;
+}
+
+// x += act · Wdᵀ; the next layer's attention norm (or the final norm) is deferred the same way.
+GemmSpec spec_down(dflash_ctx* ctx, int l, int R) {
+  const dflash_config& c = ctx->cfg;
+  GemmSpec dn;
+  dn.x = ctx->act;
+  dn.x_split = ctx->bf16;
+  dn.ldx = c.intermediate;
+  dn.M = R;
+  dn.K = c.intermediate;
+  dn.n_seg = 1;
+  dn.w[0] = ctx->wd[l];
+  dn.seg_rows[0] = c.hidden;
+  dn.tag = TAG_DOWN;
+  dn.epi.kind = EPI_RESID;
+  dn.epi.x = ctx->x;
+  dn.epi.ldx = c.hidden;
+  const bool last = l + 1 == c.n_layers;
+  dn.epi.gamma_next = last ? ctx->final_norm : ctx->attn_norm[l + 1];
+  dn.epi.out_type = OUT_BF16X2;
+  dn.epi.out_plane = (size_t)R * c.hidden;
+  dn.epi.xg = ctx->h;
+  dn.epi.sumsq = ctx->sumsq[1];
+  dn.epi.ld_part = R;
+  return dn;
+}
+
+// Final norm (deferred) -> shared LM head -> per-row argmax keys; logits are never stored.
+GemmSpec spec_lm(dflash_ctx* ctx, int R) {
+  const dflash_config& c = ctx->cfg;
+  GemmSpec lm;
+  lm.x = ctx->h;
+  // The LM head only feeds an argmax: above 32 rows it reads the hi plane alone,
+  // which halves its MMA work and activation tiles (from 64 rows on, the split
+  // makes it tensor- or shared-memory-bound). The hi plane's rounding (2^-9
+  // relative) moves a logit by ~2e-3 (std) at these scales, inside the 1e-2
+  // top-2 gap the draft tokens are held to; up to 32 rows the lo plane is free.
+  lm.x_split = ctx->bf16 && R <= 32;
+  lm.ldx = c.hidden;
+  lm.M = R;
+  lm.K = c.hidden;
+  lm.n_seg = 1;
+  lm.w[0] = ctx->lm_head;
+  lm.seg_rows[0] = c.vocab;
+  lm.tag = TAG_LM;
+  lm.epi.kind = EPI_ARGMAX;
+  lm.epi.keys = ctx->keys;
+  if (c.n_layers > 0) set_deferred_norm(ctx, lm.epi, ctx->sumsq[1], R);
+  return lm;
+}
+
 #define DFL_CHECK(call)                       \
   do {                                        \
     dflash_status s_ = (call);                \
@@ -353,6 +529,10 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     if (ctx->force_stages > 8) ctx->force_stages = 8;
     env = std::getenv("DFLASH_PDL");
     ctx->use_pdl = !(env && env[0] == '0');
+    env = std::getenv("DFLASH_ATTN");
+    ctx->attn_mma = env && std::strcmp(env, "mma") == 0;
+    env = std::getenv("DFLASH_ATTN_STAGES");
+    if (env && std::atoi(env) >= 2 && std::atoi(env) <= kMaxAttnTcStages) ctx->attn_stages = std::atoi(env);
     // Failure injection (tests only): every tensor-core GEMM epilogue gives up on a
     // barrier nothing arrives at after this many ns (capped at 100 ms), so the
     // call completes with DFLASH_ERR_TIMEOUT and no copy or MMA in flight.
@@ -669,40 +849,60 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     int kps = (std::max(max_ctx, 1) + n_splits - 1) / n_splits;
     kps = (kps + key_tile - 1) / key_tile * key_tile;
     n_splits = std::max(1, (max_ctx + kps - 1) / kps);
+    // Tensor-core (tcgen05) attention: bf16 drafter, fp16 cache, 64-key tiles that
+    // stay inside one page. One CTA per SM; the split count minimises
+    // waves x (key tiles per CTA + a fixed cost per CTA), where the resident
+    // clusters per wave come from the occupancy query (a cluster merges through
+    // distributed shared memory, at most 16 CTAs); one wave of up to one CTA per
+    // SM with a global merge is the alternative for long contexts and few pairs.
+    const bool attn_tc = ctx->bf16 && ctx->cache_f16 && !ctx->attn_mma && c.page_size % 64 == 0 && g * B <= 128 &&
+                         (c.head_dim == 64 || c.head_dim == 128);
+    if (attn_tc) {
+      const int nr = g * B;
+      const int st_n = ctx->attn_stages;
+      const int blk_tiles = (B + 63) / 64;
+      constexpr double kCtaCost = 3.0;   // fixed cost of a CTA, in key tiles
+      double best = 1e30;
+      for (int sp = 1; sp <= kMaxAttnCluster; ++sp) {
+        int kp = (std::max(max_ctx, 1) + sp - 1) / sp;
+        kp = (kp + 63) / 64 * 64;
+        if (std::max(1, (max_ctx + kp - 1) / kp) != sp) continue;
+        auto key = std::make_tuple(c.head_dim, st_n, sp, nr);
+        auto it = ctx->attn_cluster_cap.find(key);
+        const int cap = it != ctx->attn_cluster_cap.end()
+                            ? it->second
+                            : (ctx->attn_cluster_cap[key] = attn_tc_max_clusters(c.head_dim, st_n, sp, false, nr));
+        if (cap < 1) continue;
+        const double cost = (double)((pairs + cap - 1) / cap) * (kp / 64 + blk_tiles + kCtaCost);
+        if (cost < best) {
+          best = cost;
+          n_splits = sp;
+          kps = kp;
+          attn_gmerge = false;
+        }
+      }
+      // global merge: one wave, up to one CTA per SM, any split count
+      const int sp_max = std::min(ctx->num_sms / std::max(pairs, 1), (int)(ctx->att_rows / ((size_t)pairs * nr)));
+      for (int sp = kMaxAttnCluster + 1; sp <= sp_max; ++sp) {
+        int kp = (std::max(max_ctx, 1) + sp - 1) / sp;
+        kp = (kp + 63) / 64 * 64;
+        if (std::max(1, (max_ctx + kp - 1) / kp) != sp) continue;
+        const double cost = kp / 64 + blk_tiles + 2 * kCtaCost;   // + the merge kernel
+        if (cost < best) {
+          best = cost;
+          n_splits = sp;
+          kps = kp;
+          attn_gmerge = true;
+        }
+      }
+      if (best >= 1e30) return DFLASH_ERR_UNSUPPORTED;
+    }
     // split partials in global memory (CUDA-core path, or the global merge) must fit the workspace
     if ((!ctx->bf16 || attn_gmerge) && (size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows)
       return DFLASH_ERR_UNSUPPORTED;
 
     for (int l = 0; l < c.n_layers; ++l) {
-      GemmSpec qkv;
-      qkv.x = ctx->h;
-      qkv.x_split = ctx->bf16;
-      qkv.ldx = H;
-      qkv.M = R;
-      qkv.K = H;
-      qkv.n_seg = 3;
-      qkv.w[0] = ctx->wq[l];
-      qkv.w[1] = ctx->wk[l];
-      qkv.w[2] = ctx->wv[l];
-      qkv.seg_rows[0] = QD;
-      qkv.seg_rows[1] = KVD;
-      qkv.seg_rows[2] = KVD;
-      qkv.tag = TAG_QKV;
-      qkv.epi.kind = EPI_QKV;
-      qkv.epi.out_type = OUT_F16;   // the attention kernel runs in fp16
-      qkv.epi.out[0] = ctx->q;
-      qkv.epi.out[1] = ctx->kb;
-      qkv.epi.out[2] = ctx->vb;
-      qkv.epi.ld_out[0] = QD;
-      qkv.epi.ld_out[1] = KVD;
-      qkv.epi.ld_out[2] = KVD;
-      qkv.epi.rope_mask = 3u;
-      qkv.epi.head_dim = c.head_dim;
-      qkv.epi.inv_freq = ctx->inv_freq;
-      qkv.epi.rows_per_req = B;
-      qkv.epi.pos_base = d_ctx_len;
-      if (l > 0) set_deferred_norm(ctx, qkv.epi, ctx->sumsq[1], R);   // rows carry the previous layer's norm
-      DFL_CHECK(run_gemm(ctx, qkv, st));
+      DFL_CHECK(run_gemm(ctx, spec_qkv(ctx, l, R, B, d_ctx_len), st));
 
       AttnParams ap{};
       ap.q = ctx->q;
@@ -738,73 +938,33 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
         const double kvb = (double)bs * max_ctx * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;
         const double fl = 4.0 * bs * B * (double)(max_ctx + B) * QD;
         ProfScope prof(ctx, PK_ATTN, st, kvb, fl);
-        DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, hb, hb, st, ctx->use_pdl), "attention launch"));
+        if (attn_tc) {
+          AttnTcParams tp;
+          std::memset(&tp, 0, sizeof(tp));
+          tp.a = ap;
+          tp.stages = ctx->attn_stages;
+          const int D = c.head_dim;
+          const long long qd[3] = {D, c.n_q_heads, R}, qs[2] = {(long long)D * 2, (long long)QD * 2};
+          const int qb[3] = {64, g, B};
+          const long long bd[3] = {KVD, B, bs}, bst[2] = {(long long)KVD * 2, (long long)B * KVD * 2};
+          const int bb[3] = {64, 64, 1};
+          const long long cd[2] = {D, (long long)num_pages * c.n_kv_heads * c.page_size}, cst[1] = {(long long)D * 2};
+          const int cb[2] = {64, 64};
+          if (!get_map_f16(ctx, ctx->q, 3, qd, qs, qb, &tp.qmap) || !get_map_f16(ctx, ctx->kb, 3, bd, bst, bb, &tp.kbmap) ||
+              !get_map_f16(ctx, ctx->vb, 3, bd, bst, bb, &tp.vbmap) ||
+              !get_map_f16(ctx, k_cache[l], 2, cd, cst, cb, &tp.kcmap) ||
+              !get_map_f16(ctx, v_cache[l], 2, cd, cst, cb, &tp.vcmap))
+            return DFLASH_ERR_CUDA;
+          DFL_CHECK(cuda_status(launch_attn_tc(tp, ctx->ao, st, ctx->use_pdl), "attention (tcgen05) launch"));
+        } else {
+          DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, hb, hb, st, ctx->use_pdl), "attention launch"));
+        }
       }
 
-      GemmSpec o;
-      o.x = ctx->ao;
-      o.x_split = ctx->bf16;
-      o.ldx = QD;
-      o.M = R;
-      o.K = QD;
-      o.n_seg = 1;
-      o.w[0] = ctx->wo[l];
-      o.seg_rows[0] = H;
-      o.tag = TAG_O;
-      o.epi.kind = EPI_RESID;
-      o.epi.x = ctx->x;
-      o.epi.ldx = H;
-      // the MLP norm is deferred: x ⊙ gain now, the row scales in the gate/up epilogue
-      o.epi.gamma_next = ctx->mlp_norm[l];
-      o.epi.out_type = OUT_BF16X2;
-      o.epi.out_plane = (size_t)R * H;
-      o.epi.xg = ctx->h;
-      o.epi.sumsq = ctx->sumsq[0];
-      o.epi.ld_part = R;
-      DFL_CHECK(run_gemm(ctx, o, st));
-
-      GemmSpec gu;
-      gu.x = ctx->h;
-      gu.x_split = ctx->bf16;
-      gu.ldx = H;
-      gu.M = R;
-      gu.K = H;
-      gu.n_seg = 2;
-      gu.paired = true;
-      gu.w[0] = ctx->wg[l];
-      gu.w[1] = ctx->wu[l];
-      gu.seg_rows[0] = gu.seg_rows[1] = c.intermediate;
-      gu.tag = TAG_GATEUP;
-      gu.epi.kind = EPI_SWIGLU;
-      gu.epi.out_type = OUT_BF16X2;
-      gu.epi.out_plane = (size_t)R * c.intermediate;
-      gu.epi.out[0] = ctx->act;
-      gu.epi.ld_out[0] = c.intermediate;
-      set_deferred_norm(ctx, gu.epi, ctx->sumsq[0], R);
-      DFL_CHECK(run_gemm(ctx, gu, st));
-
-      GemmSpec dn;
-      dn.x = ctx->act;
-      dn.x_split = ctx->bf16;
-      dn.ldx = c.intermediate;
-      dn.M = R;
-      dn.K = c.intermediate;
-      dn.n_seg = 1;
-      dn.w[0] = ctx->wd[l];
-      dn.seg_rows[0] = H;
-      dn.tag = TAG_DOWN;
-      dn.epi.kind = EPI_RESID;
-      dn.epi.x = ctx->x;
-      dn.epi.ldx = H;
-      // the next layer's attention norm (or the final norm) is deferred the same way
+      DFL_CHECK(run_gemm(ctx, spec_o(ctx, l, R), st));
+      DFL_CHECK(run_gemm(ctx, spec_gateup(ctx, l, R), st));
+      DFL_CHECK(run_gemm(ctx, spec_down(ctx, l, R), st));
       const bool last = l + 1 == c.n_layers;
-      dn.epi.gamma_next = last ? ctx->final_norm : ctx->attn_norm[l + 1];
-      dn.epi.out_type = OUT_BF16X2;
-      dn.epi.out_plane = (size_t)R * H;
-      dn.epi.xg = ctx->h;
-      dn.epi.sumsq = ctx->sumsq[1];
-      dn.epi.ld_part = R;
-      DFL_CHECK(run_gemm(ctx, dn, st));
 
       if (d_hidden_out) {
         ProfScope prof(ctx, PK_COPY, st, (double)layer_stride * 8, 0);
@@ -825,25 +985,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
                                            ctx->use_pdl),
                             "rmsnorm launch"));
 
-    GemmSpec lm;
-    lm.x = ctx->h;
-    // The LM head only feeds an argmax: above 32 rows it reads the hi plane alone,
-    // which halves its MMA work and activation tiles (from 64 rows on, the split
-    // makes it tensor- or shared-memory-bound). The hi plane's rounding (2^-9
-    // relative) moves a logit by ~2e-3 (std) at these scales, inside the 1e-2
-    // top-2 gap the draft tokens are held to; up to 32 rows the lo plane is free.
-    lm.x_split = ctx->bf16 && R <= 32;
-    lm.ldx = H;
-    lm.M = R;
-    lm.K = H;
-    lm.n_seg = 1;
-    lm.w[0] = ctx->lm_head;
-    lm.seg_rows[0] = c.vocab;
-    lm.tag = TAG_LM;
-    lm.epi.kind = EPI_ARGMAX;
-    lm.epi.keys = ctx->keys;
-    if (c.n_layers > 0) set_deferred_norm(ctx, lm.epi, ctx->sumsq[1], R);
-    DFL_CHECK(run_gemm(ctx, lm, st));
+    DFL_CHECK(run_gemm(ctx, spec_lm(ctx, R), st));
     {
       ProfScope prof(ctx, PK_ARGMAX, st, (double)R * 8 * 2 + (double)bs * (B - 1) * 4, 0);
       const dflash_status fs = cuda_status(launch_argmax_finalize(ctx->keys, bs, B, d_draft, st, ctx->use_pdl),
@@ -856,6 +998,35 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
       }
     }
     return DFLASH_OK;
+  } catch (...) {   // no C++ exception crosses the C ABI
+    return DFLASH_ERR_OOM;
+  }
+}
+
+extern "C" dflash_status dflash_profile_gemm_chain(dflash_ctx* ctx, const void* feats, int bs, int max_new,
+                                                   const int* d_n_new, const int* d_start_pos, void* const* k_cache,
+                                                   void* const* v_cache, const int* d_page_table, int max_pages,
+                                                   int num_pages, const int* d_ctx_len, int B, void* stream) {
+  dfl::TraceRange trace_("dflash_profile_gemm_chain");
+  try {
+    if (!ctx) return DFLASH_ERR_ARG;
+    const dflash_config& c = ctx->cfg;
+    if (!ctx->bf16 || ctx->force_simt) return DFLASH_ERR_UNSUPPORTED;   // the chain times the tensor-core GEMM
+    if (bs <= 0 || bs > c.max_batch || B <= 0 || B > c.max_block || !d_ctx_len) return DFLASH_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the injection is GEMMs only: run it as dflash_inject_ctx does
+    DFL_CHECK(dflash_inject_ctx(ctx, feats, bs, max_new, d_n_new, d_start_pos, k_cache, v_cache, d_page_table,
+                                max_pages, num_pages, stream));
+    const int R = bs * B;
+    for (int l = 0; l < c.n_layers; ++l) {
+      DFL_CHECK(run_gemm(ctx, spec_qkv(ctx, l, R, B, d_ctx_len), st));
+      DFL_CHECK(run_gemm(ctx, spec_o(ctx, l, R), st));
+      DFL_CHECK(run_gemm(ctx, spec_gateup(ctx, l, R), st));
+      DFL_CHECK(run_gemm(ctx, spec_down(ctx, l, R), st));
+    }
+    DFL_CHECK(run_gemm(ctx, spec_lm(ctx, R), st));
+    // the LM head folded its maxima into the keys; the next draft must start from zero
+    return cuda_status(cudaMemsetAsync(ctx->keys, 0, (size_t)R * sizeof(unsigned long long), st), "keys reset");
   } catch (...) {   // no C++ exception crosses the C ABI
     return DFLASH_ERR_OOM;
   }

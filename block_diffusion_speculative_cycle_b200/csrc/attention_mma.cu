@@ -609,6 +609,17 @@ __global__ void __launch_bounds__(256) attn_gmerge_kernel(const AttnParams p, __
   }
 }
 
+cudaError_t launch_attn_gmerge(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {
+  const int warps = p.bs * p.B * p.n_q;
+  if (p.d == 128)
+    return launch_kernel(attn_gmerge_kernel<128>, dim3((warps + 7) / 8), dim3(256), 0, st, pdl, p,
+                         (__nv_bfloat16*)out);
+  if (p.d == 64)
+    return launch_kernel(attn_gmerge_kernel<64>, dim3((warps + 7) / 8), dim3(256), 0, st, pdl, p,
+                         (__nv_bfloat16*)out);
+  return cudaErrorInvalidValue;
+}
+
 template <int D, int NST, int KS>
 static cudaError_t launch_cluster_t(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {
   const int nr = p.g * p.B;

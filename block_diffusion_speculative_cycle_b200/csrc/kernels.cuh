@@ -37,6 +37,28 @@ struct AttnParams {
 constexpr int kMaxAttnCluster = 16;
 cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st, bool pdl);
 
+// Merge of split partials written to global memory (part_o / part_m / part_l,
+// exp2 domain) into out [R, n_q*d] as bf16 hi/lo planes (the cluster kernels'
+// global-merge mode).
+cudaError_t launch_attn_gmerge(const AttnParams& p, void* out, cudaStream_t st, bool pdl);
+
+// Tensor-core (tcgen05) attention for the bf16 drafter with an fp16 cache whose
+// page size is a multiple of 64. Tensor maps (fp16, 128-byte swizzle, boxes of
+// 64 elements inner):
+//   qmap   q [R, n_q, d] as 3D (d, n_q, R), box (64, g, B)
+//   kbmap, vbmap  block k / v [bs, B, n_kv*d] as 3D (n_kv*d, B, bs), box (64, 64, 1)
+//   kcmap, vcmap  this layer's cache pools as 2D (d, num_pages*n_kv*page_size), box (64, 64)
+constexpr int kMaxAttnTcStages = 6;
+struct alignas(64) AttnTcParams {
+  CUtensorMap qmap, kbmap, vbmap, kcmap, vcmap;
+  AttnParams a;
+  int stages;                 // K/V ring depth (2..kMaxAttnTcStages)
+};
+cudaError_t launch_attn_tc(const AttnTcParams& tp, void* out, cudaStream_t st, bool pdl);
+size_t attn_tc_smem_bytes(int d, int stages, int splits, bool gmerge, int nr);
+// Clusters of n CTAs of the tensor-core attention kernel that can be resident at once.
+int attn_tc_max_clusters(int d, int stages, int n, bool gmerge, int nr);
+
 // CUDA-core split-KV attention partials (fp32 path), then the log-sum-exp merge into out [R, n_q*d].
 cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st, bool pdl);
 

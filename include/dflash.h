@@ -239,6 +239,23 @@ dflash_status dflash_profile_enable(dflash_ctx* ctx, int enable);
  * (negative dflash_status on error). Resets the records. */
 int dflash_profile_read(dflash_ctx* ctx, dflash_profile_entry* out, int max_entries);
 
+/* GEMM-chain instrumentation, no counterpart on the pages. Enqueues on `stream`,
+ * back to back, exactly the tensor-core GEMM launches one cycle of this shape
+ * makes, with the same plans, fused epilogues and programmatic dependent
+ * launch, and nothing else: the injection's two (as dflash_inject_ctx, with the
+ * same arguments and effect on the cache), then per layer QKV, O, gate/up and
+ * down, then the LM head (R = bs * B rows, positions from d_ctx_len). Its purpose
+ * is timing the GEMMs as they run inside a cycle, overlapping each other's ramp
+ * and tail, e.g. by capturing the call in a CUDA graph and timing its replays.
+ * The draft-side results are not a draft: the context's activations and residual
+ * stream are left unspecified (the next dflash_draft_block rebuilds them) and the
+ * argmax state is cleared at the end. bf16 drafters only (DFLASH_ERR_UNSUPPORTED
+ * otherwise); argument errors as for dflash_inject_ctx / dflash_draft_block. */
+dflash_status dflash_profile_gemm_chain(dflash_ctx* ctx, const void* feats, int bs, int max_new,
+                                        const int* d_n_new, const int* d_start_pos, void* const* k_cache,
+                                        void* const* v_cache, const int* d_page_table, int max_pages, int num_pages,
+                                        const int* d_ctx_len, int B, void* stream);
+
 /* Synchronise `stream`, read and clear the context's device status word.
  * Returns DFLASH_ERR_TIMEOUT, DFLASH_ERR_DEVICE or DFLASH_OK. */
 dflash_status dflash_get_error(dflash_ctx* ctx, void* stream);

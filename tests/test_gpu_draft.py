@@ -95,3 +95,11 @@ def test_small_bf16_chunked_inject_and_padding_rows():
 def test_small_bf16_untied_head_and_many_requests():
     lens = list(np.random.default_rng(0).integers(0, 400, size=12))
     run_case(SMALL_BF16, [int(x) for x in lens], 16, seed=5, share=False)
+
+
+def test_small_bf16_fp16_cache_long_contexts():
+    """Contexts of 1000-4000 keys over 16 requests: each attention CTA streams a
+    dozen key tiles or more through its ring (wrap-around, lazy rescaling of the
+    running maximum), on the fp16 cache the tcgen05 attention kernel reads."""
+    lens = [int(x) for x in np.random.default_rng(7).integers(1000, 4001, size=16)]
+    run_case(SMALL_BF16, lens, 16, seed=9, cache_dtype=torch.float16)

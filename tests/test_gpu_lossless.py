@@ -25,13 +25,13 @@ PAGE = 64
 class GpuDrafter:
     """The library's drafter for one request, wired for oracle.target.spec_generate."""
 
-    def __init__(self, cfg, weights_cpu, max_len, B, max_inject):
+    def __init__(self, cfg, weights_cpu, max_len, B, max_inject, cache_dtype=None):
         self.cfg = cfg
         pages = (max_len + B + PAGE - 1) // PAGE
         table = torch.arange(pages, dtype=torch.int32)[None]
         self.d, _ = make_drafter(cfg, weights_cpu, max_block=B, max_batch=1, max_inject_rows=max_inject,
-                                 page_size=PAGE)
-        self.cache = PagedCache(cfg, table, pages, PAGE)
+                                 page_size=PAGE, cache_dtype=cache_dtype)
+        self.cache = PagedCache(cfg, table, pages, PAGE, dtype=cache_dtype)
         self.num_pages = pages
 
     def inject(self, feats, start):
@@ -59,6 +59,9 @@ def gpu_verify_fn(z, d):
 
 
 def run(dtype, seed, n_new, B, cheat_p=None):
+    """dtype: "f32", "bf16" (bf16 KV cache) or "bf16-f16cache" (fp16 KV cache, tcgen05 attention)."""
+    cache_dtype = torch.float16 if dtype == "bf16-f16cache" else None
+    dtype = "bf16" if cache_dtype is not None else dtype
     tw, dw = tiny_pair(seed)
     dcfg = synth.TINY if dtype == "f32" else synth.TINY.replace(dtype="bf16")
     if dtype != "f32":
@@ -68,7 +71,7 @@ def run(dtype, seed, n_new, B, cheat_p=None):
     prompt = synth.make_tokens(TARGET_CFG, 64, seed=50 + seed).tolist()
     tgt = T.TinyTarget(TARGET_CFG, tw, n_feat=3, max_len=64 + n_new + B + 1)
     ref = T.greedy_decode(tgt, prompt, n_new)
-    drafter = GpuDrafter(dcfg, dw, 64 + n_new + B + 1, B, max_inject=64)
+    drafter = GpuDrafter(dcfg, dw, 64 + n_new + B + 1, B, max_inject=64, cache_dtype=cache_dtype)
     draft_fn = drafter.draft
     if cheat_p is not None:
         rng = np.random.default_rng(seed)
@@ -87,13 +90,13 @@ def run(dtype, seed, n_new, B, cheat_p=None):
     return out, ref, stats["accepted"]
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "bf16-f16cache"])
 def test_gpu_spec_decode_is_lossless(dtype):
     out, ref, _ = run(dtype, 0, 96, 4)
     assert out == ref
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "bf16-f16cache"])
 def test_gpu_spec_decode_lossless_at_every_acceptance_length(dtype):
     out, ref, acc = run(dtype, 2, 128, 4, cheat_p=0.75)
     assert out == ref
