@@ -432,7 +432,7 @@ def run_ours(args, world, rank, local):
     dflash_profile_enable(c.drafter.handle, False)
     prof.append({"name": "verify", "launches": args.profile_steps, "total_ms": v_ms,
                  "bytes": args.profile_steps * (c.bs * c.B * c.cfg.vocab * 2 + c.bs * c.B * 8.0), "flops": 0.0})
-    kernels_per_cycle = sum(e["launches"] * (2 if e["name"] == "attention" else 1) for e in prof) / args.profile_steps
+    kernels_per_cycle = sum(e["launches"] for e in prof) / args.profile_steps
 
     # the dominant kernel: GEMM call sites share one kernel, so they are summed
     kinds = {}

@@ -184,8 +184,8 @@ def dflash_profile_enable(handle, enable: bool) -> None:
 def dflash_profile_read(handle) -> List[dict]:
     """Aggregated per-kernel timings since the last read: list of dicts
     (name, launches, total_ms, bytes, flops)."""
-    arr = (dflash_profile_entry * 16)()
-    n = load_library().dflash_profile_read(handle, arr, 16)
+    arr = (dflash_profile_entry * 32)()
+    n = load_library().dflash_profile_read(handle, arr, 32)
     if n < 0:
         raise DFlashError(-n, "dflash_profile_read")
     return [{"name": arr[i].name.decode(), "launches": arr[i].launches, "total_ms": arr[i].total_ms,

@@ -33,6 +33,7 @@ enum ProfKind {
   PK_GEMM_TC = 0,                    // + tag
   PK_GEMM_SIMT = PK_GEMM_TC + TAG_COUNT,   // + tag
   PK_ATTN = PK_GEMM_SIMT + TAG_COUNT,
+  PK_ATTN_MERGE,
   PK_EMBED_NORM,
   PK_RMSNORM,
   PK_ARGMAX,
@@ -42,7 +43,7 @@ enum ProfKind {
 const char* const kProfNames[PK_COUNT] = {
     "gemm_tc:fc", "gemm_tc:kv", "gemm_tc:qkv", "gemm_tc:o", "gemm_tc:gateup", "gemm_tc:down", "gemm_tc:lm",
     "gemm_simt:fc", "gemm_simt:kv", "gemm_simt:qkv", "gemm_simt:o", "gemm_simt:gateup", "gemm_simt:down",
-    "gemm_simt:lm", "attention", "embed_norm", "rmsnorm", "argmax_finalize", "hidden_copy"};
+    "gemm_simt:lm", "attention", "attention_merge", "embed_norm", "rmsnorm", "argmax_finalize", "hidden_copy"};
 
 struct ProfRec {
   int kind;
@@ -64,7 +65,9 @@ struct dflash_ctx {
   int split_slots = 2;    // CTAs per SM the K-split plan fills (DFLASH_SPLIT_SLOTS, experiments)
   unsigned test_stall_ns = 0;   // DFLASH_TEST_STALL_NS: failure-injection hook of the tensor-core GEMM
   bool attn_mma = false;        // DFLASH_ATTN=mma: the mma.sync attention kernel even where tcgen05 applies
-  int attn_stages = 4;          // K/V ring depth of the tcgen05 attention (DFLASH_ATTN_STAGES, experiments)
+  int attn_form = -1;           // DFLASH_ATTN_FORM=full|compact: force the tcgen05 attention form (experiments)
+  int attn_l2promo = 3;         // DFLASH_ATTN_L2PROMO=0..3: L2 promotion of the attention's tensor maps (experiments)
+  int attn_stages = 5;          // K/V ring depth of the tcgen05 attention (DFLASH_ATTN_STAGES, experiments)
   std::map<std::tuple<int, int, int, int>, int> attn_cluster_cap;   // resident clusters per (d, stages, n, rows)
   int num_sms = 148;
   const void* fc = nullptr;
@@ -178,9 +181,12 @@ bool get_map_f16(dflash_ctx* ctx, const void* ptr, int rank, const long long* di
   }
   for (int i = 0; i + 1 < rank; ++i) st[i] = (cuuint64_t)strides[i];
   CUtensorMap m;
+  static const CUtensorMapL2promotion promo[4] = {CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_64B,
+                                                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B};
   CUresult r = ctx->encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), d, st, bx,
-                           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo[ctx->attn_l2promo],
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     std::fprintf(stderr, "dflash: tensor map encode failed (%d)\n", (int)r);
     return false;
@@ -531,8 +537,13 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     ctx->use_pdl = !(env && env[0] == '0');
     env = std::getenv("DFLASH_ATTN");
     ctx->attn_mma = env && std::strcmp(env, "mma") == 0;
+    env = std::getenv("DFLASH_ATTN_FORM");
+    if (env) ctx->attn_form = std::strcmp(env, "compact") == 0 ? 1 : (std::strcmp(env, "full") == 0 ? 0 : -1);
+    env = std::getenv("DFLASH_ATTN_L2PROMO");
+    if (env && std::atoi(env) >= 0 && std::atoi(env) <= 3) ctx->attn_l2promo = std::atoi(env);
     env = std::getenv("DFLASH_ATTN_STAGES");
     if (env && std::atoi(env) >= 2 && std::atoi(env) <= kMaxAttnTcStages) ctx->attn_stages = std::atoi(env);
+    if (c.head_dim == 128 && ctx->attn_stages > 5) ctx->attn_stages = 5;   // what fits beside Q and P
     // Failure injection (tests only): every tensor-core GEMM epilogue gives up on a
     // barrier nothing arrives at after this many ns (capped at 100 ms), so the
     // call completes with DFLASH_ERR_TIMEOUT and no copy or MMA in flight.
@@ -850,53 +861,78 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
     kps = (kps + key_tile - 1) / key_tile * key_tile;
     n_splits = std::max(1, (max_ctx + kps - 1) / kps);
     // Tensor-core (tcgen05) attention: bf16 drafter, fp16 cache, 64-key tiles that
-    // stay inside one page. One CTA per SM; the split count minimises
-    // waves x (key tiles per CTA + a fixed cost per CTA), where the resident
-    // clusters per wave come from the occupancy query (a cluster merges through
-    // distributed shared memory, at most 16 CTAs); one wave of up to one CTA per
-    // SM with a global merge is the alternative for long contexts and few pairs.
+    // stay inside one page. Two forms: full (one CTA per SM, a ring of
+    // attn_stages K/V tiles) and compact (two CTAs per SM, two stages each). For
+    // the chosen form the split count minimises waves x CTA time, a CTA's time in
+    // units of one key tile being a start-up (first HBM round trip, merge) plus
+    // its tiles (the rate a lone CTA sustains is set by its S -> softmax -> P·V
+    // chain, not by HBM),
+    // where the clusters resident per wave come from the occupancy query (a
+    // cluster merges through distributed shared memory, at most 16 CTAs), or uses
+    // one wave of CTAs with a global merge (a second kernel) and any split count.
     const bool attn_tc = ctx->bf16 && ctx->cache_f16 && !ctx->attn_mma && c.page_size % 64 == 0 && g * B <= 128 &&
                          (c.head_dim == 64 || c.head_dim == 128);
+    bool attn_compact = false;
     if (attn_tc) {
       const int nr = g * B;
-      const int st_n = ctx->attn_stages;
       const int blk_tiles = (B + 63) / 64;
-      constexpr double kCtaCost = 3.0;   // fixed cost of a CTA, in key tiles
+      // Form: with few (request, KV head) pairs the full form's deeper pipeline wins;
+      // from 16 pairs on, two CTAs per SM hide each other's per-tile chain (both
+      // measured on B200 across the benchmark workloads).
+      const int want_form = ctx->attn_form >= 0 ? ctx->attn_form : (pairs >= 16 ? 1 : 0);
+      constexpr double kStart = 4.0, kMergeKernel = 3.0;
       double best = 1e30;
-      for (int sp = 1; sp <= kMaxAttnCluster; ++sp) {
-        int kp = (std::max(max_ctx, 1) + sp - 1) / sp;
-        kp = (kp + 63) / 64 * 64;
-        if (std::max(1, (max_ctx + kp - 1) / kp) != sp) continue;
-        auto key = std::make_tuple(c.head_dim, st_n, sp, nr);
-        auto it = ctx->attn_cluster_cap.find(key);
-        const int cap = it != ctx->attn_cluster_cap.end()
-                            ? it->second
-                            : (ctx->attn_cluster_cap[key] = attn_tc_max_clusters(c.head_dim, st_n, sp, false, nr));
-        if (cap < 1) continue;
-        const double cost = (double)((pairs + cap - 1) / cap) * (kp / 64 + blk_tiles + kCtaCost);
-        if (cost < best) {
-          best = cost;
-          n_splits = sp;
-          kps = kp;
-          attn_gmerge = false;
+      for (int form = 0; form < 2; ++form) {
+        const bool compact = form == 1;
+        if (form != want_form) continue;
+        const int st_n = compact ? 2 : ctx->attn_stages;
+        const double t_tile = compact ? 1.25 : 1.0;
+        for (int sp = 1; sp <= kMaxAttnCluster; ++sp) {
+          int kp = (std::max(max_ctx, 1) + sp - 1) / sp;
+          kp = (kp + 63) / 64 * 64;
+          if (std::max(1, (max_ctx + kp - 1) / kp) != sp) continue;
+          auto key = std::make_tuple(c.head_dim * 2 + (int)compact, st_n, sp, nr);
+          auto it = ctx->attn_cluster_cap.find(key);
+          const int cap =
+              it != ctx->attn_cluster_cap.end()
+                  ? it->second
+                  : (ctx->attn_cluster_cap[key] = attn_tc_max_clusters(c.head_dim, compact, st_n, sp, false, nr));
+          if (ctx->debug && sp <= 4) std::fprintf(stderr, "dflash attention form %d cluster %d: %d resident\n", form, sp, cap);
+          if (cap < 1) continue;
+          const double cost = (double)((pairs + cap - 1) / cap) * (kStart + (kp / 64 + blk_tiles) * t_tile);
+          if (cost < best) {
+            best = cost;
+            n_splits = sp;
+            kps = kp;
+            attn_gmerge = false;
+            attn_compact = compact;
+          }
         }
-      }
-      // global merge: one wave, up to one CTA per SM, any split count
-      const int sp_max = std::min(ctx->num_sms / std::max(pairs, 1), (int)(ctx->att_rows / ((size_t)pairs * nr)));
-      for (int sp = kMaxAttnCluster + 1; sp <= sp_max; ++sp) {
-        int kp = (std::max(max_ctx, 1) + sp - 1) / sp;
-        kp = (kp + 63) / 64 * 64;
-        if (std::max(1, (max_ctx + kp - 1) / kp) != sp) continue;
-        const double cost = kp / 64 + blk_tiles + 2 * kCtaCost;   // + the merge kernel
-        if (cost < best) {
-          best = cost;
-          n_splits = sp;
-          kps = kp;
-          attn_gmerge = true;
+        // global merge: every CTA resident at once, any split count
+        const int per_sm = compact ? 2 : 1;
+        const int sp_max =
+            std::min(per_sm * ctx->num_sms / std::max(pairs, 1), (int)(ctx->att_rows / ((size_t)pairs * nr)));
+        for (int sp = 2; sp <= sp_max; ++sp) {
+          int kp = (std::max(max_ctx, 1) + sp - 1) / sp;
+          kp = (kp + 63) / 64 * 64;
+          if (std::max(1, (max_ctx + kp - 1) / kp) != sp) continue;
+          const double cost = kStart + kMergeKernel + (kp / 64 + blk_tiles) * t_tile;
+          if (cost < best) {
+            best = cost;
+            n_splits = sp;
+            kps = kp;
+            attn_gmerge = true;
+            attn_compact = compact;
+          }
         }
       }
       if (best >= 1e30) return DFLASH_ERR_UNSUPPORTED;
     }
+    if (ctx->debug)
+      std::fprintf(stderr, "dflash attention %s%s pairs=%d splits=%d kps=%d gmerge=%d max_ctx=%d\n",
+                   attn_tc ? "tcgen05" : (ctx->bf16 ? "mma.sync" : "simt"), attn_compact ? " compact" : "", pairs,
+                   n_splits, kps, (int)attn_gmerge,
+                   max_ctx);
     // split partials in global memory (CUDA-core path, or the global merge) must fit the workspace
     if ((!ctx->bf16 || attn_gmerge) && (size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows)
       return DFLASH_ERR_UNSUPPORTED;
@@ -943,6 +979,7 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
           std::memset(&tp, 0, sizeof(tp));
           tp.a = ap;
           tp.stages = ctx->attn_stages;
+          tp.compact = attn_compact ? 1 : 0;
           const int D = c.head_dim;
           const long long qd[3] = {D, c.n_q_heads, R}, qs[2] = {(long long)D * 2, (long long)QD * 2};
           const int qb[3] = {64, g, B};
@@ -959,6 +996,12 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
         } else {
           DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, hb, hb, st, ctx->use_pdl), "attention launch"));
         }
+      }
+      if (attn_tc && attn_gmerge) {
+        // partials: n_splits x (O, m, l) per query row, read once; the output rows (two planes)
+        const double pb = (double)bs * c.n_kv_heads * n_splits * g * B * (c.head_dim + 2) * 4 + (double)R * QD * 2 * es;
+        ProfScope prof2(ctx, PK_ATTN_MERGE, st, pb, 0);
+        DFL_CHECK(cuda_status(launch_attn_gmerge(ap, ctx->ao, st, ctx->use_pdl), "attention merge launch"));
       }
 
       DFL_CHECK(run_gemm(ctx, spec_o(ctx, l, R), st));

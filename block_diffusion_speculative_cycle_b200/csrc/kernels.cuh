@@ -52,12 +52,14 @@ constexpr int kMaxAttnTcStages = 6;
 struct alignas(64) AttnTcParams {
   CUtensorMap qmap, kbmap, vbmap, kcmap, vcmap;
   AttnParams a;
-  int stages;                 // K/V ring depth (2..kMaxAttnTcStages)
+  int stages;                 // K/V ring depth of the full form (2..kMaxAttnTcStages; 5 fits with d = 128)
+  int compact;                // the compact form: <= 64 query rows, two-stage ring, two CTAs per SM
 };
+// With a.global_merge set, the caller follows it with launch_attn_gmerge.
 cudaError_t launch_attn_tc(const AttnTcParams& tp, void* out, cudaStream_t st, bool pdl);
-size_t attn_tc_smem_bytes(int d, int stages, int splits, bool gmerge, int nr);
-// Clusters of n CTAs of the tensor-core attention kernel that can be resident at once.
-int attn_tc_max_clusters(int d, int stages, int n, bool gmerge, int nr);
+size_t attn_tc_smem_bytes(int d, bool compact, int stages, int splits, bool gmerge, int nr);
+// Clusters of n CTAs (n = 1: single CTAs) of the tensor-core attention kernel that can be resident at once.
+int attn_tc_max_clusters(int d, bool compact, int stages, int n, bool gmerge, int nr);
 
 // CUDA-core split-KV attention partials (fp32 path), then the log-sum-exp merge into out [R, n_q*d].
 cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st, bool pdl);
