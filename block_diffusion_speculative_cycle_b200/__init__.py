@@ -9,5 +9,6 @@ from ._binding import (  # noqa: F401
     DFLASH_BF16, DFLASH_F16, DFLASH_F32, DFlashError, Drafter, dflash_create, dflash_destroy, dflash_draft_block,
     dflash_get_error, dflash_inject_ctx, dflash_profile_enable, dflash_profile_gemm_chain, dflash_profile_read,
     dflash_status_string, dflash_verify, dflash_verify_workspace_size,
-    exported_symbols, load_library, verify,
+    dflash_draft_block_sample, dflash_verify_sampled, dflash_verify_sampled_workspace_size,
+    exported_symbols, load_library, verify, verify_sampled,
 )

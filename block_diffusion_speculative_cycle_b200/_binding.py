@@ -21,7 +21,8 @@ DFLASH_F16 = 2
 _STATUS = {0: "DFLASH_OK", 1: "DFLASH_ERR_ARG", 2: "DFLASH_ERR_CUDA", 3: "DFLASH_ERR_OOM",
            4: "DFLASH_ERR_TIMEOUT", 5: "DFLASH_ERR_DEVICE", 6: "DFLASH_ERR_UNSUPPORTED"}
 
-EXPORTS = ["dflash_create", "dflash_destroy", "dflash_inject_ctx", "dflash_draft_block",
+EXPORTS = ["dflash_create", "dflash_destroy", "dflash_inject_ctx", "dflash_draft_block", "dflash_draft_block_sample",
+           "dflash_verify_sampled_workspace_size", "dflash_verify_sampled",
            "dflash_verify_workspace_size", "dflash_verify", "dflash_verify_noalloc", "dflash_profile_enable", "dflash_profile_read",
            "dflash_profile_gemm_chain", "dflash_get_error", "dflash_status_string"]
 
@@ -77,6 +78,14 @@ def load_library(path: Optional[str] = None):
     lib.dflash_inject_ctx.restype = c_int
     lib.dflash_draft_block.argtypes = [_P, _P, _P, c_int, c_int, _PP, _PP, _P, c_int, c_int, c_int, _P, _P, _P]
     lib.dflash_draft_block.restype = c_int
+    lib.dflash_draft_block_sample.argtypes = [_P, _P, _P, c_int, c_int, _PP, _PP, _P, c_int, c_int, c_int,
+                                              ctypes.c_float, ctypes.c_ulonglong, _P, _P, _P, _P]
+    lib.dflash_draft_block_sample.restype = c_int
+    lib.dflash_verify_sampled_workspace_size.argtypes = [c_int, c_int, c_int]
+    lib.dflash_verify_sampled_workspace_size.restype = c_size
+    lib.dflash_verify_sampled.argtypes = [_P, c_int, _P, _P, c_int, c_int, c_int, ctypes.c_float, _P, _P, _P, _P, _P,
+                                          c_size, _P]
+    lib.dflash_verify_sampled.restype = c_int
     lib.dflash_verify_workspace_size.argtypes = [c_int, c_int]
     lib.dflash_verify_workspace_size.restype = c_size
     lib.dflash_verify.argtypes = [_P, c_int, _P, c_int, c_int, c_int, _P, _P, _P, c_size, _P]
@@ -161,6 +170,44 @@ def dflash_draft_block(handle, anchor, ctx_len, bs, B, k_cache, v_cache, page_ta
     _check(lib.dflash_draft_block(handle, _ptr(anchor), _ptr(ctx_len), bs, B, _ptr_array(k_cache),
                                   _ptr_array(v_cache), _ptr(page_table), page_table.shape[1], num_pages, max_ctx,
                                   _ptr(draft), _ptr(hidden_out), _stream(stream)), "dflash_draft_block")
+
+
+def dflash_draft_block_sample(handle, anchor, ctx_len, bs, B, k_cache, v_cache, page_table, num_pages, max_ctx,
+                              temperature, seed, draft, draft_logits, hidden_out=None, stream=None) -> None:
+    lib = load_library()
+    _check(lib.dflash_draft_block_sample(handle, _ptr(anchor), _ptr(ctx_len), bs, B, _ptr_array(k_cache),
+                                         _ptr_array(v_cache), _ptr(page_table), page_table.shape[1], num_pages,
+                                         max_ctx, float(temperature), int(seed), _ptr(draft), _ptr(draft_logits),
+                                         _ptr(hidden_out), _stream(stream)), "dflash_draft_block_sample")
+
+
+def dflash_verify_sampled_workspace_size(bs: int, B: int, V: int) -> int:
+    return int(load_library().dflash_verify_sampled_workspace_size(bs, B, V))
+
+
+def dflash_verify_sampled(logits, draft_logits, draft, temperature, u_accept, u_final, accepted, next_token,
+                          workspace, stream=None) -> None:
+    import torch
+    lib = load_library()
+    bs, B, V = logits.shape
+    dt = DFLASH_BF16 if logits.dtype == torch.bfloat16 else DFLASH_F32
+    _check(lib.dflash_verify_sampled(_ptr(logits), dt, _ptr(draft_logits), _ptr(draft), bs, B, V, float(temperature),
+                                     _ptr(u_accept), _ptr(u_final), _ptr(accepted), _ptr(next_token),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "dflash_verify_sampled")
+
+
+def verify_sampled(logits, draft_logits, draft, temperature, u_accept, u_final, workspace=None, stream=None):
+    """Allocate outputs (and scratch unless given) and run dflash_verify_sampled; returns (accepted, next_token)."""
+    import torch
+    bs, B, V = logits.shape
+    dev = logits.device
+    acc = torch.empty(bs, dtype=torch.int32, device=dev)
+    nxt = torch.empty(bs, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.zeros(dflash_verify_sampled_workspace_size(bs, B, V), dtype=torch.uint8, device=dev)
+    dflash_verify_sampled(logits, draft_logits, draft, temperature, u_accept, u_final, acc, nxt, workspace, stream)
+    return acc, nxt
 
 
 def dflash_verify_workspace_size(bs: int, B: int) -> int:
@@ -272,6 +319,11 @@ class Drafter:
               hidden_out=None, stream=None):
         dflash_draft_block(self.handle, anchor, ctx_len, bs, B, k_cache, v_cache, page_table, num_pages, max_ctx,
                            draft, hidden_out, stream)
+
+    def draft_sample(self, anchor, ctx_len, bs, B, k_cache, v_cache, page_table, num_pages, max_ctx, temperature, seed,
+                     draft, draft_logits, hidden_out=None, stream=None):
+        dflash_draft_block_sample(self.handle, anchor, ctx_len, bs, B, k_cache, v_cache, page_table, num_pages,
+                                  max_ctx, temperature, seed, draft, draft_logits, hidden_out, stream)
 
     def check(self, stream=None):
         st = dflash_get_error(self.handle, stream)

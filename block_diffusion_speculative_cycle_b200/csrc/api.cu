@@ -794,11 +794,20 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
   }
 }
 
-extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_len, int bs,
-                                            int B, const void* const* k_cache, const void* const* v_cache,
-                                            const int* d_page_table, int max_pages, int num_pages, int max_ctx,
-                                            int* d_draft, float* d_hidden_out, void* stream) {
-  dfl::TraceRange trace_("dflash_draft_block");
+namespace {
+
+// Sampled drafting (temperature > 0): the LM head draws each draft token by the
+// Gumbel-max rule and stores the drafter's logits for the sampled verify.
+struct SampleArgs {
+  float inv_temp;
+  uint32_t seed_lo, seed_hi;
+  float* logits_out;
+};
+
+dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_len, int bs, int B,
+                         const void* const* k_cache, const void* const* v_cache, const int* d_page_table,
+                         int max_pages, int num_pages, int max_ctx, int* d_draft, float* d_hidden_out, void* stream,
+                         const SampleArgs* smp) {
   try {
     if (!ctx) return DFLASH_ERR_ARG;
     const dflash_config& c = ctx->cfg;
@@ -1028,7 +1037,19 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
                                            ctx->use_pdl),
                             "rmsnorm launch"));
 
-    DFL_CHECK(run_gemm(ctx, spec_lm(ctx, R), st));
+    {
+      GemmSpec lm = spec_lm(ctx, R);
+      if (smp) {
+        lm.epi.kind = EPI_SAMPLE;
+        lm.epi.inv_temp = smp->inv_temp;
+        lm.epi.seed_lo = smp->seed_lo;
+        lm.epi.seed_hi = smp->seed_hi;
+        lm.epi.logits_out = smp->logits_out;
+        lm.epi.ld_logits = c.vocab;
+        lm.epi.rows_per_req = B;
+      }
+      DFL_CHECK(run_gemm(ctx, lm, st));
+    }
     {
       ProfScope prof(ctx, PK_ARGMAX, st, (double)R * 8 * 2 + (double)bs * (B - 1) * 4, 0);
       const dflash_status fs = cuda_status(launch_argmax_finalize(ctx->keys, bs, B, d_draft, st, ctx->use_pdl),
@@ -1044,6 +1065,36 @@ extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor
   } catch (...) {   // no C++ exception crosses the C ABI
     return DFLASH_ERR_OOM;
   }
+}
+
+}  // namespace
+
+extern "C" dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_len, int bs,
+                                            int B, const void* const* k_cache, const void* const* v_cache,
+                                            const int* d_page_table, int max_pages, int num_pages, int max_ctx,
+                                            int* d_draft, float* d_hidden_out, void* stream) {
+  dfl::TraceRange trace_("dflash_draft_block");
+  return draft_impl(ctx, d_anchor, d_ctx_len, bs, B, k_cache, v_cache, d_page_table, max_pages, num_pages, max_ctx,
+                    d_draft, d_hidden_out, stream, nullptr);
+}
+
+extern "C" dflash_status dflash_draft_block_sample(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_len,
+                                                   int bs, int B, const void* const* k_cache,
+                                                   const void* const* v_cache, const int* d_page_table,
+                                                   int max_pages, int num_pages, int max_ctx, float temperature,
+                                                   unsigned long long seed, int* d_draft, float* d_draft_logits,
+                                                   float* d_hidden_out, void* stream) {
+  dfl::TraceRange trace_("dflash_draft_block_sample");
+  if (!ctx) return DFLASH_ERR_ARG;
+  if (!(temperature > 0.f) || !std::isfinite(temperature)) return DFLASH_ERR_ARG;
+  if (B > 1 && !d_draft_logits) return DFLASH_ERR_ARG;
+  SampleArgs smp;
+  smp.inv_temp = 1.0f / temperature;
+  smp.seed_lo = (uint32_t)(seed & 0xffffffffull);
+  smp.seed_hi = (uint32_t)(seed >> 32);
+  smp.logits_out = d_draft_logits;
+  return draft_impl(ctx, d_anchor, d_ctx_len, bs, B, k_cache, v_cache, d_page_table, max_pages, num_pages, max_ctx,
+                    d_draft, d_hidden_out, stream, &smp);
 }
 
 extern "C" dflash_status dflash_profile_gemm_chain(dflash_ctx* ctx, const void* feats, int bs, int max_new,

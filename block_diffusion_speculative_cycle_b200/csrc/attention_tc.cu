@@ -26,11 +26,11 @@
 //              TMEM lane) and 64/WPQ of the tile's key columns; it reads them with
 //              tcgen05.ld, the row's maximum is combined across the WPQ threads
 //              of the row through shared memory, and it keeps a running max and
-//              sum in the exp2 domain and writes its part of P (fp16) to shared
-//              memory in the MMA's swizzled K-major layout. The running max is
-//              raised lazily: only when a row's max grows by more than 2^8 is O
-//              rescaled in TMEM (tcgen05.ld / st) and the sum with it, so P stays
-//              <= 2^8 in fp16.
+//              sum in the exp2 domain and writes its part of P (fp16 pairs) back
+//              over the tile's S in TMEM (tcgen05.st), where the P·V MMA reads its
+//              A operand. The running max is raised lazily: only when a row's max
+//              grows by more than 2^8 is O rescaled in TMEM (tcgen05.ld / st) and
+//              the sum with it, so P stays <= 2^8 in fp16.
 // After the last tile the rows' (O, m, l) are merged across the splits of the
 // (request, head): through distributed shared memory inside a cluster, or, for
 // many splits, through global memory and a second kernel. Every wait is bounded;
@@ -80,8 +80,8 @@ __device__ __forceinline__ int p_rows_of(const AttnTcParams& tp) { return tp.a.g
 // follows and give TMEM lanes 64..127, which nothing reads); otherwise, and in the
 // full form (one CTA per SM, `stages` stages, 4 S/P buffers, 16 softmax warps),
 // Q is zero-padded to 128 rows.
-// Either way one P buffer: the softmax of tile t writes it once the P·V of tile
-// t-1 has read it, which the MMA issues as soon as that P is complete.
+// The S buffer of tile t is reused for tile t + NSB once the P·V of tile t (which
+// reads P from it) has completed; the MMA issues each P·V as soon as its P is complete.
 template <int D, bool COMPACT>
 __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
     attn_tc_kernel(const __grid_constant__ AttnTcParams tp, __nv_bfloat16* out) {

@@ -7,6 +7,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "philox.cuh"
 
 namespace dfl {
 
@@ -22,6 +23,7 @@ enum EpiKind : int {
   EPI_RESID = 3,      // x[m, n] += acc                                  (Wo, Wdown)
   EPI_SWIGLU = 4,     // act[m, f] = silu(gate) * up (paired gate/up tiles)
   EPI_ARGMAX = 5,     // per activation row, max over the tile's vocab rows -> keys[m]
+  EPI_SAMPLE = 6,     // Gumbel-max draw per row (keys[m]) + the row's logits stored
 };
 
 struct EpiParams {
@@ -54,6 +56,13 @@ struct EpiParams {
   void* xg;
   float* sumsq;
   unsigned long long* keys;          // [M] packed argmax keys
+  // EPI_SAMPLE: row m = request m / rows_per_req, block position i = m % rows_per_req;
+  // rows with i >= 1 draw argmax_v (logit / T + Gumbel noise) into keys[m] and store
+  // their logits (fp32) at logits_out[(req * (rows_per_req - 1) + i - 1) * ld_logits + v].
+  float inv_temp;
+  uint32_t seed_lo, seed_hi;
+  float* logits_out;
+  int ld_logits;
   int* status;
   int out_type;                      // OUT_F32 / OUT_BF16 / OUT_F16 / OUT_BF16X2 (see store_out)
   size_t out_plane;                  // OUT_BF16X2: elements from the hi plane to the lo plane
@@ -223,6 +232,34 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
       const float g = A(j, c), u = A(j, c + kTileN / 2);
       store_out(e.out[0], (size_t)(row0 + j) * e.ld_out[0] + f, silu_f(g) * u, e.out_type, e.out_plane);
     }
+  } else if constexpr (KIND == EPI_SAMPLE) {
+    // warp w takes rows w, w+4, ...; lane scans vocab rows vbase + lane + 32k, k < 4,
+    // whose uniforms are the four words of one Philox block at counter
+    // (tile, lane, i, req): the draft-noise layout of the sampled drafter
+    const int w = t >> 5, lane = t & 31;
+    const int vbase = tile * kTileN;
+#pragma unroll 1
+    for (int j = w; j < nrows; j += 4) {
+      const int m = row0 + j;
+      const int req = m / e.rows_per_req, i = m % e.rows_per_req;
+      if (i == 0) continue;   // the anchor row drafts nothing
+      const uint4 r = philox4x32_10(make_uint4((uint32_t)tile, (uint32_t)lane, (uint32_t)i, (uint32_t)req), e.seed_lo,
+                                    e.seed_hi);
+      const uint32_t words[4] = {r.x, r.y, r.z, r.w};
+      float* lo = e.logits_out + ((size_t)req * (e.rows_per_req - 1) + i - 1) * e.ld_logits + vbase;
+      unsigned long long best = 0ull;
+#pragma unroll
+      for (int k = 0; k < kTileN / 32; ++k) {
+        const int c = lane + 32 * k;
+        const float logit = A(j, c);
+        lo[c] = logit;
+        const float gumbel = -logf(-logf(philox_uniform(words[k])));
+        const unsigned long long key = argmax_key(fmaf(logit, e.inv_temp, gumbel), vbase + c);
+        best = key > best ? key : best;
+      }
+      best = warp_max_u64(best);
+      if (lane == 0) atomicMax(e.keys + m, best);
+    }
   } else if constexpr (KIND == EPI_ARGMAX) {
     // warp w takes rows w, w+4, ...; each lane scans 4 of the tile's 128 vocab rows
     const int w = t >> 5, lane = t & 31;
@@ -255,6 +292,7 @@ __device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, in
     case EPI_RESID: epilogue_chunk_k<EPI_RESID>(e, tile, row0, nrows, acc, t, rs, red); break;
     case EPI_SWIGLU: epilogue_chunk_k<EPI_SWIGLU>(e, tile, row0, nrows, acc, t, rs, red); break;
     case EPI_ARGMAX: epilogue_chunk_k<EPI_ARGMAX>(e, tile, row0, nrows, acc, t, rs, red); break;
+    case EPI_SAMPLE: epilogue_chunk_k<EPI_SAMPLE>(e, tile, row0, nrows, acc, t, rs, red); break;
     default: break;
   }
 }

@@ -288,9 +288,10 @@ cudaError_t launch_gemm_tc(const GemmTcParams& p, cudaStream_t st) {
     case EPI_RESID: kernel = (const void*)gemm_tc_kernel<EPI_RESID>; break;
     case EPI_SWIGLU: kernel = (const void*)gemm_tc_kernel<EPI_SWIGLU>; break;
     case EPI_ARGMAX: kernel = (const void*)gemm_tc_kernel<EPI_ARGMAX>; break;
+    case EPI_SAMPLE: kernel = (const void*)gemm_tc_kernel<EPI_SAMPLE>; break;
     default: return cudaErrorInvalidValue;
   }
-  static size_t attr_bytes[EPI_ARGMAX + 1] = {};
+  static size_t attr_bytes[EPI_SAMPLE + 1] = {};
   if (smem > attr_bytes[p.epi.kind]) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -171,6 +171,24 @@ dflash_status dflash_draft_block(dflash_ctx* ctx, const int* d_anchor, const int
                                  const int* d_page_table, int max_pages, int num_pages, int max_ctx,
                                  int* d_draft, float* d_hidden_out, void* stream);
 
+/* Sampled drafting (temperature T > 0; [P1] §1 speculative sampling, [P2] results
+ * at temperature 1): the same drafter pass as dflash_draft_block, but each draft
+ * token is drawn from softmax(logits_i / T) by the Gumbel-max rule,
+ *   d_i = argmax_v (logits_i[v] / T - log(-log u_i[v])),
+ * fused into the LM head, and the drafter's logits are stored for the sampled
+ * verify (its q). The uniforms are Philox4x32-10 (Salmon et al., SC 2011) under
+ * key `seed`: for request r, position i (1..B-1) and vocabulary entry v, word
+ * (v mod 128) div 32 of the block at counter (v div 128, v mod 32, i, r), mapped
+ * to ((word >> 9) + 1/2) / 2^23. Pass a new seed per cycle for independent draws.
+ *   temperature    > 0 and finite (DFLASH_ERR_ARG otherwise)
+ *   d_draft_logits [bs, B-1, V] fp32 (device, out): logits of positions 1..B-1
+ * Other arguments, outputs and errors as for dflash_draft_block. */
+dflash_status dflash_draft_block_sample(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_len, int bs, int B,
+                                        const void* const* k_cache, const void* const* v_cache,
+                                        const int* d_page_table, int max_pages, int num_pages, int max_ctx,
+                                        float temperature, unsigned long long seed, int* d_draft,
+                                        float* d_draft_logits, float* d_hidden_out, void* stream);
+
 /* Bytes of scratch dflash_verify needs for (bs, B). */
 size_t dflash_verify_workspace_size(int bs, int B);
 
@@ -191,6 +209,32 @@ size_t dflash_verify_workspace_size(int bs, int B);
 dflash_status dflash_verify(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft,
                             int bs, int B, int V, int* d_accepted, int* d_next_token,
                             void* d_workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of scratch dflash_verify_sampled needs for (bs, B, V). */
+size_t dflash_verify_sampled_workspace_size(int bs, int B, int V);
+
+/* Sampled verify (T > 0; [P1] §1: keep drafts the target agrees with, from the
+ * first rejection draw from the target, so the output follows target-only
+ * sampling; the standard speculative-sampling rule, position by position).
+ * With p_j = softmax(logits[r, j] / T) and q_i = softmax(draft_logits[r, i-1] / T):
+ *   draft i (1..B-1) is accepted while u_accept[r, i-1] * q_i(d_i) < p_{i-1}(d_i);
+ *   a_r = the number accepted; next_r is drawn from max(0, p_a - q_{a+1}),
+ *   normalised (p_a itself if that is zero everywhere), or from p_{B-1} when every
+ *   draft passed: the smallest v whose running sum in index order exceeds
+ *   u_final[r] times the total.
+ *   d_logits       [bs, B, V] target logits in logits_dtype (bf16 or fp32)
+ *   d_draft_logits [bs, B-1, V] fp32: the drafter's logits (dflash_draft_block_sample)
+ *   d_draft        [bs, B-1] int32; an id outside [0, V) is rejected
+ *   d_u_accept     [bs, B-1] fp32, d_u_final [bs] fp32: uniforms in [0, 1) (inputs)
+ *   d_workspace    at least dflash_verify_sampled_workspace_size(bs, B, V) bytes,
+ *                  256-byte aligned, zero-filled before its first use; every call
+ *                  leaves the part that must start at zero zeroed again. Calls that
+ *                  share a workspace must not overlap on the GPU.
+ * Computed in fp32 with every sum in a fixed order: reproducible run to run. */
+dflash_status dflash_verify_sampled(const void* d_logits, dflash_dtype logits_dtype, const float* d_draft_logits,
+                                    const int* d_draft, int bs, int B, int V, float temperature,
+                                    const float* d_u_accept, const float* d_u_final, int* d_accepted,
+                                    int* d_next_token, void* d_workspace, size_t workspace_bytes, void* stream);
 
 /* Verify for callers that cannot allocate device memory. Same computation,
  * outputs and bit-exact results as dflash_verify; the pages have no

@@ -10,8 +10,8 @@ Modules
   dflash  -- feature fusion + KV injection, the block drafter, greedy verify
   target  -- a tiny causal target model, greedy autoregressive decoding and the
              speculative loop (for the lossless check)
-  sampling -- sampled (temperature > 0) verification and Gumbel-max drafting,
-             the groundwork for the sampled-verify kernel (no CUDA counterpart yet)
+  sampling -- sampled (temperature > 0) verification and Gumbel-max drafting
+  philox  -- the Philox4x32-10 counter-based generator of the draft noise
 
 Parity status per function (what pins each one, see tests/test_oracle_*.py):
   rms_norm, silu, apply_rope, block_attention, drafter_layer, inject,
@@ -21,6 +21,8 @@ Parity status per function (what pins each one, see tests/test_oracle_*.py):
   spec_generate               pinned (library decoder, lossless invariant)
   softmax_t, sample_index,
   sampled_verify,
-  gumbel_sample               pinned (exact first-token marginal, special cases,
+  gumbel_sample, gumbel_draft pinned (exact first-token marginal, special cases,
                               greedy limit, Markov-chain loop, softmax frequencies)
+  philox4x32_10, draft_uniforms
+                              pinned (published known-answer vectors, layout, moments)
 """

@@ -11,6 +11,10 @@ Sources (page title, section):
   [P2] "한 번에 초안을 생성하는 DFlash ..." (results): the speed-up holds with
        sampling at temperature 1, not only for greedy decoding.
 
+The sampled drafter draws its tokens with gumbel_draft: the Gumbel-max rule over
+the counter-based uniforms of oracle.philox (the CUDA side generates the same
+stream from the same published generator).
+
 Reading (the pages name the scheme but print no formula): the standard
 speculative-sampling rule, position by position over the block. Draft d_i was
 drawn from the drafter's distribution q_i (the block drafter predicts every
@@ -27,6 +31,8 @@ from __future__ import annotations
 from typing import Sequence, Tuple
 
 import numpy as np
+
+from .philox import draft_uniforms
 
 
 def softmax_t(logits, temperature: float) -> np.ndarray:
@@ -77,3 +83,21 @@ def gumbel_sample(logits, temperature: float, u) -> np.ndarray:
     z = np.asarray(logits, dtype=np.float64) / float(temperature)
     g = -np.log(-np.log(np.asarray(u, dtype=np.float64)))
     return np.argmax(z + g, axis=-1)
+
+
+def gumbel_draft(logits, temperature: float, seed: int, b: int) -> np.ndarray:
+    """The sampled drafter's tokens for request b: row i-1 of logits [B-1, V] holds
+    the drafter's logits at block position i, and d_i is their Gumbel-max draw
+    with the Philox draft-noise uniforms of (seed, b, i) (oracle.philox)."""
+    logits = np.asarray(logits, dtype=np.float64)
+    Bm1, V = logits.shape
+    u = np.stack([draft_uniforms(seed, b, i, V) for i in range(1, Bm1 + 1)]) if Bm1 else np.zeros((0, V))
+    return gumbel_sample(logits, temperature, u)
+
+
+def gumbel_scores(logits, temperature: float, seed: int, b: int) -> np.ndarray:
+    """The perturbed scores logits / T - log(-log u) that gumbel_draft maximises."""
+    logits = np.asarray(logits, dtype=np.float64)
+    Bm1, V = logits.shape
+    u = np.stack([draft_uniforms(seed, b, i, V) for i in range(1, Bm1 + 1)])
+    return logits / float(temperature) - np.log(-np.log(u))

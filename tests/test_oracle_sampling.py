@@ -132,3 +132,19 @@ def test_gumbel_max_draws_follow_the_softmax():
     np.testing.assert_allclose(freq, S.softmax_t(logits, T)[0], atol=8e-3)
     # vanishing temperature: the argmax
     assert (S.gumbel_sample(np.repeat(logits, 100, 0), 1e-6, rng.random(size=(100, 4))) == 2).all()
+
+
+def test_gumbel_draft_uses_the_philox_stream_and_follows_softmax():
+    """gumbel_draft is the Gumbel-max rule over the Philox draft uniforms: its
+    token at position i maximises the perturbed scores, and over many requests
+    (independent streams) the draws follow softmax(logits / T)."""
+    from oracle import philox as X
+    rng = np.random.default_rng(5)
+    logits = rng.normal(size=(3, 6))
+    d = S.gumbel_draft(logits, 0.8, seed=99, b=2)
+    for i in range(1, 4):
+        u = X.draft_uniforms(99, 2, i, 6)
+        assert d[i - 1] == int(np.argmax(logits[i - 1] / 0.8 - np.log(-np.log(u))))
+    draws = np.array([S.gumbel_draft(logits[:1], 0.8, seed=7, b=b)[0] for b in range(20000)])
+    freq = np.bincount(draws, minlength=6) / draws.size
+    np.testing.assert_allclose(freq, S.softmax_t(logits[:1], 0.8)[0], atol=0.012)
