@@ -38,7 +38,7 @@ class dflash_config(ctypes.Structure):
         "hidden", "n_layers", "n_q_heads", "n_kv_heads", "head_dim", "intermediate", "vocab", "n_feat_layers",
         "target_hidden", "mask_token_id", "max_block", "max_batch", "max_inject_rows", "page_size")] + [
         ("rope_theta", ctypes.c_float), ("rms_eps", ctypes.c_float), ("dtype", ctypes.c_int),
-        ("cache_dtype", ctypes.c_int)]
+        ("cache_dtype", ctypes.c_int), ("window", ctypes.c_int)]
 
 
 _P = ctypes.c_void_p
@@ -274,7 +274,7 @@ class Drafter:
     weights: dict with fc, embed, lm_head, final_norm and per-layer dicts (see synth)."""
 
     def __init__(self, cfg, weights: Dict, max_block: int, max_batch: int = 1, max_inject_rows: int = 64,
-                 page_size: int = 64, cache_dtype=None):
+                 page_size: int = 64, cache_dtype=None, window: int = 0):
         import torch
         self.cfg = cfg
         self.weights = weights
@@ -287,6 +287,7 @@ class Drafter:
         c.dtype = DFLASH_BF16 if cfg.dtype == "bf16" else DFLASH_F32
         # KV cache element type: the model dtype unless fp16 is asked for (bf16 drafters)
         c.cache_dtype = DFLASH_F16 if cache_dtype == torch.float16 else c.dtype
+        c.window = window
         self.cache_dtype = torch.float16 if cache_dtype == torch.float16 else cfg.torch_dtype
         self.config = c
         L = weights["layers"]

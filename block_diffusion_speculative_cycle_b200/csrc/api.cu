@@ -501,6 +501,7 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
         c.max_batch <= 0 || c.max_inject_rows < 0 || c.page_size <= 0 || !(c.rope_theta > 0.f) || !(c.rms_eps >= 0.f))
       return DFLASH_ERR_ARG;
     if (c.mask_token_id < 0 || c.mask_token_id >= c.vocab) return DFLASH_ERR_ARG;
+    if (c.window < 0) return DFLASH_ERR_ARG;
     if (c.n_q_heads % c.n_kv_heads) return DFLASH_ERR_ARG;
     if (c.dtype != DFLASH_F32 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
     if (c.cache_dtype == DFLASH_F16 && c.dtype != DFLASH_BF16) return DFLASH_ERR_ARG;
@@ -848,7 +849,10 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
     const int g = c.n_q_heads / c.n_kv_heads;
     const int pairs = bs * c.n_kv_heads;
     const int key_tile = ctx->bf16 ? 64 : 32;
-    const int ctx_tiles = std::max(1, (max_ctx + key_tile - 1) / key_tile);
+    // keys a request's block can attend to: the whole context, or with a sliding
+    // window at most window + 63 from the window's 64-aligned start
+    const int span = c.window > 0 ? std::min(max_ctx, c.window + 63) : max_ctx;
+    const int ctx_tiles = std::max(1, (span + key_tile - 1) / key_tile);
     int attn_ks = 1, n_splits;
     bool attn_gmerge = false;
     if (ctx->bf16) {
@@ -866,9 +870,9 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
     } else {
       n_splits = std::max(1, (kAttnTargetCtas + pairs - 1) / pairs);
     }
-    int kps = (std::max(max_ctx, 1) + n_splits - 1) / n_splits;
+    int kps = (std::max(span, 1) + n_splits - 1) / n_splits;
     kps = (kps + key_tile - 1) / key_tile * key_tile;
-    n_splits = std::max(1, (max_ctx + kps - 1) / kps);
+    n_splits = std::max(1, (span + kps - 1) / kps);
     // Tensor-core (tcgen05) attention: bf16 drafter, fp16 cache, 64-key tiles that
     // stay inside one page. Two forms: full (one CTA per SM, a ring of
     // attn_stages K/V tiles) and compact (two CTAs per SM, two stages each). For
@@ -897,9 +901,9 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
         const int st_n = compact ? 2 : ctx->attn_stages;
         const double t_tile = compact ? 1.25 : 1.0;
         for (int sp = 1; sp <= kMaxAttnCluster; ++sp) {
-          int kp = (std::max(max_ctx, 1) + sp - 1) / sp;
+          int kp = (std::max(span, 1) + sp - 1) / sp;
           kp = (kp + 63) / 64 * 64;
-          if (std::max(1, (max_ctx + kp - 1) / kp) != sp) continue;
+          if (std::max(1, (span + kp - 1) / kp) != sp) continue;
           auto key = std::make_tuple(c.head_dim * 2 + (int)compact, st_n, sp, nr);
           auto it = ctx->attn_cluster_cap.find(key);
           const int cap =
@@ -922,9 +926,9 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
         const int sp_max =
             std::min(per_sm * ctx->num_sms / std::max(pairs, 1), (int)(ctx->att_rows / ((size_t)pairs * nr)));
         for (int sp = 2; sp <= sp_max; ++sp) {
-          int kp = (std::max(max_ctx, 1) + sp - 1) / sp;
+          int kp = (std::max(span, 1) + sp - 1) / sp;
           kp = (kp + 63) / 64 * 64;
-          if (std::max(1, (max_ctx + kp - 1) / kp) != sp) continue;
+          if (std::max(1, (span + kp - 1) / kp) != sp) continue;
           const double cost = kStart + kMergeKernel + (kp / 64 + blk_tiles) * t_tile;
           if (cost < best) {
             best = cost;
@@ -938,10 +942,9 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
       if (best >= 1e30) return DFLASH_ERR_UNSUPPORTED;
     }
     if (ctx->debug)
-      std::fprintf(stderr, "dflash attention %s%s pairs=%d splits=%d kps=%d gmerge=%d max_ctx=%d\n",
+      std::fprintf(stderr, "dflash attention %s%s pairs=%d splits=%d kps=%d gmerge=%d span=%d\n",
                    attn_tc ? "tcgen05" : (ctx->bf16 ? "mma.sync" : "simt"), attn_compact ? " compact" : "", pairs,
-                   n_splits, kps, (int)attn_gmerge,
-                   max_ctx);
+                   n_splits, kps, (int)attn_gmerge, span);
     // split partials in global memory (CUDA-core path, or the global merge) must fit the workspace
     if ((!ctx->bf16 || attn_gmerge) && (size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows)
       return DFLASH_ERR_UNSUPPORTED;
@@ -971,6 +974,7 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
       ap.ks = attn_ks;
       ap.global_merge = attn_gmerge ? 1 : 0;
       ap.max_ctx = max_ctx;
+      ap.window = c.window;
       ap.scale = (float)(1.0 / std::sqrt((double)c.head_dim));
       ap.part_o = ctx->att_o;
       ap.part_m = ctx->att_m;
@@ -980,8 +984,8 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
       ap.cache_f16 = ctx->cache_f16 ? 1 : 0;
       {
         // context K/V of every request (upper bound max_ctx), block q/k/v, output
-        const double kvb = (double)bs * max_ctx * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;
-        const double fl = 4.0 * bs * B * (double)(max_ctx + B) * QD;
+        const double kvb = (double)bs * span * KVD * 2 * es + (double)R * (2 * QD + 2 * KVD) * es;
+        const double fl = 4.0 * bs * B * (double)(span + B) * QD;
         ProfScope prof(ctx, PK_ATTN, st, kvb, fl);
         if (attn_tc) {
           AttnTcParams tp;

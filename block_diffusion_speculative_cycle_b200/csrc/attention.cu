@@ -36,7 +36,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
     P = P < 0 ? 0 : p.max_ctx;
   }
   const int T_all = P + p.B;
-  const int k0 = s * p.kps, k1 = s == p.n_splits - 1 ? T_all : min(T_all, k0 + p.kps);
+  const int ctx_lo = attn_ctx_lo(P, p.window);
+  const int k0 = min(T_all, attn_key_base(ctx_lo) + s * p.kps),
+            k1 = s == p.n_splits - 1 ? T_all : min(T_all, k0 + p.kps);
 
   for (int e = threadIdx.x; e < nr * D; e += kAttnThreads) {
     const int r = e / D, dd = e % D, j = r / p.B, i = r % p.B;
@@ -56,7 +58,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
     for (int e = threadIdx.x; e < kKeyTile * D; e += kAttnThreads) {
       const int kk = e / D, dd = e % D, key = kt + kk;
       float kv = 0.f, vv = 0.f;
-      if (key < k1) {
+      if (key < k1 && key >= ctx_lo) {
         if (key < P) {
           const int slot = key / p.page_size;
           const int page = slot < p.max_pages ? p.page_table[(size_t)b * p.max_pages + slot] : -1;
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
       vs[kk * (D + 1) + dd] = vv;
     }
     __syncthreads();
-    const bool valid = kt + lane < k1;
+    const bool valid = kt + lane < k1 && kt + lane >= ctx_lo;
 #pragma unroll
     for (int rr = 0; rr < RPW; ++rr) {
       const int r = warp + 8 * rr;
@@ -91,7 +93,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
         }
         const float mn = fmaxf(m[rr], warp_max(sc));
         const float pe = valid ? expf(sc - mn) : 0.f;
-        const float alpha = expf(m[rr] - mn);
+        // a tile with every key masked (below a sliding window's start) while the
+        // row has seen no key yet leaves the state as it is
+        const float alpha = mn == -INFINITY ? 1.f : expf(m[rr] - mn);
         l[rr] = l[rr] * alpha + warp_sum(pe);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) o[rr][c] *= alpha;
@@ -138,7 +142,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p, OT*
   const int nr = p.g * p.B, r = jj * p.B + i;
   int P = p.ctx_len[b];
   P = P < 0 ? 0 : (P > p.max_ctx ? p.max_ctx : P);
-  const int used = min(p.n_splits, (P + p.B + p.kps - 1) / p.kps);
+  const int used = min(p.n_splits, (P + p.B - attn_key_base(attn_ctx_lo(P, p.window)) + p.kps - 1) / p.kps);
   const size_t base = (size_t)(b * p.n_kv + h) * p.n_splits * nr + r;
   float M = -INFINITY;
   for (int s = lane; s < used; s += 32) M = fmaxf(M, p.part_m[base + (size_t)s * nr]);

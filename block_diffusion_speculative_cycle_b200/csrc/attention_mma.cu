@@ -133,9 +133,12 @@ __global__ void __launch_bounds__(KS == 2 ? 512 : 256, KS == 2 ? 1 : 0) attn_clu
     P = P < 0 ? 0 : p.max_ctx;
   }
   const int T_all = P + p.B;
-  // split s takes keys [s*kps, (s+1)*kps); the last split also takes the rest
-  // (the block keys of the longest requests run up to B past n_splits*kps)
-  const int k0 = s * p.kps, k1 = s == p.n_splits - 1 ? T_all : min(T_all, k0 + p.kps);
+  // split s takes keys [base + s*kps, base + (s+1)*kps) (base: the 64-aligned start
+  // of a sliding window, else 0); the last split also takes the rest (the block
+  // keys of the longest requests run up to B past that); keys below ctx_lo are masked
+  const int ctx_lo = attn_ctx_lo(P, p.window);
+  const int k0 = min(T_all, attn_key_base(ctx_lo) + s * p.kps),
+            k1 = s == p.n_splits - 1 ? T_all : min(T_all, k0 + p.kps);
   const int n_tiles = k1 > k0 ? (k1 - k0 + kKT - 1) / kKT : 0;
 
   const int S = p.n_splits;
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(KS == 2 ? 512 : 256, KS == 2 ? 1 : 0) attn_clu
       const void* ksrc = kb;
       const void* vsrc = vb;
       int bytes = 0;
-      if (key < k1) {
+      if (key < k1 && key >= ctx_lo) {
         if (key < P) {
           const int slot = key / p.page_size;
           const int page = slot < p.max_pages ? p.page_table[(size_t)b * p.max_pages + slot] : -1;
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(KS == 2 ? 512 : 256, KS == 2 ? 1 : 0) attn_clu
         const int key = kt + n * 8 + 2 * tig;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const bool ok = key + c < k1;
+          const bool ok = key + c < k1 && key + c >= ctx_lo;
           sc[n][c] = ok ? sc[n][c] * sl2 : -INFINITY;
           sc[n][2 + c] = ok ? sc[n][2 + c] * sl2 : -INFINITY;
           mx0 = fmaxf(mx0, sc[n][c]);
@@ -568,7 +571,7 @@ __global__ void __launch_bounds__(256) attn_gmerge_kernel(const AttnParams p, __
   const int nr = p.g * p.B, r = jj * p.B + i;
   int P = p.ctx_len[b];
   P = P < 0 ? 0 : (P > p.max_ctx ? p.max_ctx : P);
-  const int used = min(p.n_splits, (P + p.B + p.kps - 1) / p.kps);
+  const int used = min(p.n_splits, (P + p.B - attn_key_base(attn_ctx_lo(P, p.window)) + p.kps - 1) / p.kps);
   const size_t base = (size_t)(b * p.n_kv + h) * p.n_splits * nr + r;
   float M = -INFINITY;
   for (int s = lane; s < used; s += 32) M = fmaxf(M, __ldcg(p.part_m + base + (size_t)s * nr));

@@ -126,10 +126,13 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
     if (threadIdx.x == 0) flag_error(status, ST_BAD_CTX);
     P = P < 0 ? 0 : p.max_ctx;
   }
-  // this split's keys: [k0, k1) of the sequence (P context keys, then B block keys)
+  // this split's keys: [k0, k1) of the sequence (P context keys, then B block keys),
+  // counted from the 64-aligned start of a sliding window (else from 0); context
+  // keys below ctx_lo are masked
   const int S = p.n_splits;
   const int T_all = P + p.B;
-  const int k0 = min(T_all, s * p.kps);
+  const int ctx_lo = attn_ctx_lo(P, p.window);
+  const int k0 = min(T_all, attn_key_base(ctx_lo) + s * p.kps);
   const int k1 = s == S - 1 ? T_all : min(T_all, k0 + p.kps);
   const int cx1 = min(k1, P);                               // context part [k0, cx1)
   const int n_ctx = cx1 > k0 ? (cx1 - k0 + kKT - 1) / kKT : 0;
@@ -139,6 +142,8 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
   auto tile_valid = [&](int t) {
     return t < n_ctx ? min(kKT, cx1 - (k0 + t * kKT)) : min(kKT, bk1 - (bk0 + (t - n_ctx) * kKT));
   };
+  // first valid key column of a tile (non-zero only for the tile holding ctx_lo)
+  auto tile_lo = [&](int t) { return t < n_ctx ? max(0, ctx_lo - (k0 + t * kKT)) : 0; };
 
   const bool gmerge = p.global_merge != 0;
   if (gmerge && n_tiles == 0) return;   // nothing of this request here: the merge kernel skips the split
@@ -337,6 +342,7 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
       if (ok) ok = !s_abort && mbar_wait(&s_full[t % NSB], (t / NSB) & 1, status);
       const bool wok = __all_sync(0xffffffffu, ok);
       const int valid = tile_valid(t);
+      const int vlo = tile_lo(t);
       float sv[SC];   // raw scores; the max is taken before scaling (sl2 > 0)
       float mx = -INFINITY;
       if (wok && quad_live) {
@@ -344,12 +350,13 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
         uint32_t sr[SC];
         tmem_ld_cols<SC>(lane_addr + (uint32_t)((t % NSB) * kKT + c0), sr);
         tmem_wait_ld();
-        if (valid >= c0 + SC) {
+        if (valid >= c0 + SC && vlo <= c0) {
 #pragma unroll
           for (int c = 0; c < SC; ++c) sv[c] = __uint_as_float(sr[c]);
         } else {
 #pragma unroll
-          for (int c = 0; c < SC; ++c) sv[c] = c0 + c < valid ? __uint_as_float(sr[c]) : -INFINITY;
+          for (int c = 0; c < SC; ++c)
+            sv[c] = c0 + c < valid && c0 + c >= vlo ? __uint_as_float(sr[c]) : -INFINITY;
         }
         float m8[8];
 #pragma unroll
@@ -418,17 +425,18 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
         tmem_wait_st();
         l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       }
-      // a partial tile: V rows past the valid keys may hold anything (even NaN,
+      // a partial tile: V rows outside the valid keys may hold anything (even NaN,
       // which a zero probability would not cancel); zero them
-      if (valid < kKT) {
+      if (valid < kKT || vlo > 0) {
         uint8_t* vd = ring + (size_t)(t % NST) * STAGE + HALVES * KH;
-        const int n = (kKT - valid) * 8;
+        const int n_hi = (kKT - valid) * 8, n = n_hi + vlo * 8;   // 16-byte chunks per column block
         for (int e = tid; e < n * HALVES; e += kSoftThreads) {
           const int hh = e / n, c = e % n;
-          *reinterpret_cast<uint4*>(vd + hh * KH + valid * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          const int off = c < n_hi ? valid * 128 + c * 16 : (c - n_hi) * 16;
+          *reinterpret_cast<uint4*>(vd + hh * KH + off) = make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();   // the zeroed V rows, for the MMA
       }
-      if (valid < kKT) fence_proxy_async_smem();   // the zeroed V rows, for the MMA
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t % NSB]);

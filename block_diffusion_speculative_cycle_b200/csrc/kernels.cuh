@@ -27,7 +27,14 @@ struct AttnParams {
   size_t out_plane;           // tensor-core path: elements from the output's hi plane to its lo plane
   int cache_f16;              // tensor-core path: the cache pools hold fp16 (else bf16, converted on load)
   int global_merge;           // tensor-core path: splits write part_o/m/l (exp2 domain) and a second kernel merges
+  int window;                 // sliding window: the block sees context positions P-window .. P-1 only (0: all)
 };
+
+// First context key the block attends to, and the 64-aligned key where split 0
+// starts (keys from there up to ctx_lo are masked; a 64-key tile never crosses a
+// page of a multiple of 64 keys, so the tile stays inside ctx_lo's page).
+__device__ __forceinline__ int attn_ctx_lo(int P, int window) { return window > 0 ? max(0, P - window) : 0; }
+__device__ __forceinline__ int attn_key_base(int ctx_lo) { return ctx_lo & ~63; }
 
 // Tensor-core attention for the bf16 drafter (q / block k / block v fp16, cache bf16 or fp16):
 // the n_splits CTAs of one (request, KV head) form a cluster and merge through

@@ -91,6 +91,13 @@ typedef struct {
    * other value means "same as dtype" (so a zero-initialised field keeps the
    * model dtype). DFLASH_F16 with an fp32 drafter is rejected (DFLASH_ERR_ARG). */
   dflash_dtype cache_dtype;
+  /* Sliding window of the drafter's attention over its cache ("DFlash 소개": the
+   * MLX backend bounds the drafter KV cache by a sliding window for long inputs):
+   * with window W > 0 the block of a request with context length P attends to
+   * context positions max(0, P - W) .. P-1 only (and to the whole block), and
+   * never reads the cache below them, so pages that hold only older positions
+   * may be released and their page-table slots left as -1. 0: no window. */
+  int window;
 } dflash_config;
 
 /* Weights: device pointers, [out_features, in_features] row-major, in

@@ -20,7 +20,9 @@ Readings where the pages are silent (each the plainest one the rest of the pages
   * drafter layer = pre-norm RMSNorm (gain, eps) -> GQA attention with
     rotate-half RoPE -> residual; RMSNorm -> SwiGLU MLP -> residual;
     q head j reads kv head floor(j / (n_q / n_kv)); softmax scale 1/sqrt(d);
-  * argmax: lowest index among equal maxima, NaN ranks below every number.
+  * argmax: lowest index among equal maxima, NaN ranks below every number;
+  * a sliding window of W positions keeps the last W context positions
+    (P-W .. P-1) visible to the block, with their original (absolute) RoPE.
 
 Everything is computed in float64 from the inputs as given (bf16 inputs are
 widened exactly); nothing is rounded in between.
@@ -169,23 +171,34 @@ def drafter_layer(cfg, lw: Dict, x: np.ndarray, pos: np.ndarray, k_ctx: np.ndarr
     return x
 
 
+def window_start(P: int, window: int) -> int:
+    """First context position a block at P attends to: P - window for a sliding
+    window of `window` positions ("DFlash 소개": the MLX backend bounds the
+    drafter's KV cache by a sliding window for long contexts), 0 without one
+    (window 0)."""
+    return max(0, P - window) if window > 0 else 0
+
+
 def draft_block(cfg, weights: Dict, anchor: int, cache: Cache, B: int,
-                ctx_len: Optional[int] = None) -> Dict[str, object]:
+                ctx_len: Optional[int] = None, window: int = 0) -> Dict[str, object]:
     """One non-autoregressive drafter pass ([P1] §2 cycle steps 1-3; [P3] §2.2).
 
     Block = the anchor (last accepted token) at position P, then B-1 mask tokens
     at P+1..P+B-1; all B-1 masked positions are predicted in this single pass
-    through the shared, frozen embedding and LM head ([P3] §2.3).
+    through the shared, frozen embedding and LM head ([P3] §2.3). With a sliding
+    window (window > 0) the block attends to context positions
+    window_start(P, window) .. P-1 only; the block itself is always fully visible.
 
     Returns dict(draft [B-1] int, logits [B-1, V] float64, hidden: list of the
     residual stream after every layer [B, H] plus the final normed rows)."""
     P = cache.length if ctx_len is None else ctx_len
+    lo = window_start(P, window)
     ids = [int(anchor)] + [cfg.mask_token_id] * (B - 1)
     x = f64(weights["embed"])[ids]
     pos = np.arange(P, P + B)
     hidden = []
     for l, lw in enumerate(weights["layers"]):
-        x = drafter_layer(cfg, lw, x, pos, cache.k[l][:P], cache.v[l][:P])
+        x = drafter_layer(cfg, lw, x, pos, cache.k[l][lo:P], cache.v[l][lo:P])
         hidden.append(x)
     y = rms_norm(x, weights["final_norm"], cfg.rms_eps)
     hidden.append(y)

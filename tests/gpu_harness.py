@@ -70,7 +70,8 @@ def gather_cpu_cache(cfg, pools_cpu, table_cpu: torch.Tensor, r: int, P: int, pa
     return O.Cache.from_arrays(cfg, ks, vs)
 
 
-def make_drafter(cfg, weights_cpu, max_block, max_batch=1, max_inject_rows=64, page_size=64, cache_dtype=None):
+def make_drafter(cfg, weights_cpu, max_block, max_batch=1, max_inject_rows=64, page_size=64, cache_dtype=None,
+                 window=0):
     wd = to_dev(weights_cpu)
     return Drafter(cfg, wd, max_block=max_block, max_batch=max_batch, max_inject_rows=max_inject_rows,
-                   page_size=page_size, cache_dtype=cache_dtype), wd
+                   page_size=page_size, cache_dtype=cache_dtype, window=window), wd

@@ -103,3 +103,55 @@ def test_small_bf16_fp16_cache_long_contexts():
     running maximum), on the fp16 cache the tcgen05 attention kernel reads."""
     lens = [int(x) for x in np.random.default_rng(7).integers(1000, 4001, size=16)]
     run_case(SMALL_BF16, lens, 16, seed=9, cache_dtype=torch.float16)
+
+
+@pytest.mark.parametrize("cfg,cache_dtype", [(synth.TINY, None), (SMALL_BF16, None), (SMALL_BF16, torch.float16)],
+                         ids=["fp32-simt", "bf16-mma", "fp16-tcgen05"])
+@pytest.mark.parametrize("window", [128, 100])
+def test_sliding_window_matches_the_oracle_with_released_pages(cfg, cache_dtype, window):
+    """Sliding-window drafting: each request's block sees its last `window` context
+    positions. After injection the page-table slots wholly below every window are
+    set to -1 (pages released): the pass must not read them, flag nothing, and
+    match the oracle's windowed pass."""
+    ctx_lens, B, page = [300, 50, 700, 129], 16, 64
+    bs = len(ctx_lens)
+    ctx = torch.tensor(ctx_lens, dtype=torch.int32)
+    w = synth.make_drafter_weights(cfg, seed=8, share_embed_lm_head=False)
+    table, num_pages = synth.make_page_table(ctx, page, extra_tokens=B, seed=9)
+    max_new = max(ctx_lens)
+    feats = synth.make_features(cfg, bs * max_new, seed=10).reshape(bs, max_new, cfg.feat_dim)
+    anchors = synth.make_tokens(cfg, bs, seed=11)
+    drafter, _ = make_drafter(cfg, w, max_block=B, max_batch=bs, max_inject_rows=bs * max_new, page_size=page,
+                              cache_dtype=cache_dtype, window=window)
+    cache = PagedCache(cfg, table, num_pages, page, dtype=cache_dtype)
+    n_new = torch.tensor(ctx_lens, dtype=torch.int32, device="cuda")
+    start = torch.zeros(bs, dtype=torch.int32, device="cuda")
+    drafter.inject(feats.cuda(), bs, max_new, n_new, start, cache.k, cache.v, cache.table, num_pages)
+    drafter.check()
+    released = table.clone()
+    for r, P in enumerate(ctx_lens):
+        lo = O.window_start(P, window)
+        released[r, : lo // page] = -1
+    assert int((released < 0).sum()) > int((table < 0).sum())   # some pages are gone
+    draft = torch.zeros((bs, B - 1), dtype=torch.int32, device="cuda")
+    hidden = torch.zeros((cfg.n_layers + 1, bs, B, cfg.hidden), dtype=torch.float32, device="cuda")
+    drafter.draft(anchors.cuda(), ctx.cuda(), bs, B, cache.k, cache.v, released.cuda(), num_pages, max(ctx_lens),
+                  draft, hidden)
+    drafter.check()   # no page outside the windows was touched
+    draft, hidden = draft.cpu().numpy(), hidden.cpu().numpy()
+    tol = TOL[cfg.dtype]
+    moved = 0.0
+    for r, P in enumerate(ctx_lens):
+        oc = O.Cache(cfg)
+        oc.write(0, O.inject(cfg, w, feats[r, :P], 0)[1])
+        ref = O.draft_block(cfg, w, int(anchors[r]), oc, B, window=window)
+        for l in range(cfg.n_layers + 1):
+            err = max_abs_rel(hidden[l, r], ref["hidden"][l])
+            assert err <= tol, f"request {r} layer {l}: max-abs-rel {err:.3g}"
+        sure = top2_gap(ref["logits"]) > 1e-2
+        np.testing.assert_array_equal(draft[r][sure], ref["draft"][sure])
+        if P > window:
+            full = O.draft_block(cfg, w, int(anchors[r]), oc, B)
+            moved = max(moved, max_abs_rel(full["hidden"][-1], ref["hidden"][-1]))
+    assert moved > 2 * tol   # the window changes the pass well beyond the bar (the check has teeth)
+    drafter.close()

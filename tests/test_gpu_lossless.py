@@ -25,12 +25,12 @@ PAGE = 64
 class GpuDrafter:
     """The library's drafter for one request, wired for oracle.target.spec_generate."""
 
-    def __init__(self, cfg, weights_cpu, max_len, B, max_inject, cache_dtype=None):
+    def __init__(self, cfg, weights_cpu, max_len, B, max_inject, cache_dtype=None, window=0):
         self.cfg = cfg
         pages = (max_len + B + PAGE - 1) // PAGE
         table = torch.arange(pages, dtype=torch.int32)[None]
         self.d, _ = make_drafter(cfg, weights_cpu, max_block=B, max_batch=1, max_inject_rows=max_inject,
-                                 page_size=PAGE, cache_dtype=cache_dtype)
+                                 page_size=PAGE, cache_dtype=cache_dtype, window=window)
         self.cache = PagedCache(cfg, table, pages, PAGE, dtype=cache_dtype)
         self.num_pages = pages
 
@@ -58,7 +58,7 @@ def gpu_verify_fn(z, d):
     return int(acc.item()), int(nxt.item())
 
 
-def run(dtype, seed, n_new, B, cheat_p=None):
+def run(dtype, seed, n_new, B, cheat_p=None, window=0):
     """dtype: "f32", "bf16" (bf16 KV cache) or "bf16-f16cache" (fp16 KV cache, tcgen05 attention)."""
     cache_dtype = torch.float16 if dtype == "bf16-f16cache" else None
     dtype = "bf16" if cache_dtype is not None else dtype
@@ -71,7 +71,7 @@ def run(dtype, seed, n_new, B, cheat_p=None):
     prompt = synth.make_tokens(TARGET_CFG, 64, seed=50 + seed).tolist()
     tgt = T.TinyTarget(TARGET_CFG, tw, n_feat=3, max_len=64 + n_new + B + 1)
     ref = T.greedy_decode(tgt, prompt, n_new)
-    drafter = GpuDrafter(dcfg, dw, 64 + n_new + B + 1, B, max_inject=64, cache_dtype=cache_dtype)
+    drafter = GpuDrafter(dcfg, dw, 64 + n_new + B + 1, B, max_inject=64, cache_dtype=cache_dtype, window=window)
     draft_fn = drafter.draft
     if cheat_p is not None:
         rng = np.random.default_rng(seed)
@@ -101,3 +101,12 @@ def test_gpu_spec_decode_lossless_at_every_acceptance_length(dtype):
     out, ref, acc = run(dtype, 2, 128, 4, cheat_p=0.75)
     assert out == ref
     assert set(acc) == {0, 1, 2, 3}
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16-f16cache"])
+def test_gpu_spec_decode_with_a_sliding_window_drafter_is_lossless(dtype):
+    """A drafter that sees only the last 48 context positions proposes differently,
+    but the output is still the target's own greedy decode."""
+    out, ref, acc = run(dtype, 3, 128, 4, cheat_p=0.5, window=48)
+    assert out == ref
+    assert len(set(acc)) > 1

@@ -166,3 +166,76 @@ def test_attention_to_context_depends_on_relative_position_only():
     for l, lw in enumerate(w["layers"]):
         x = O.drafter_layer(cfg, lw, x, np.arange(49, 52), shifted[l][0], shifted[l][1])
     np.testing.assert_allclose(x, r0["hidden"][cfg.n_layers - 1], rtol=1e-9, atol=1e-10)
+
+
+# --------------------------------------------------------------------------- sliding window
+
+def _window_case(seed=0, P=40, B=4):
+    from block_diffusion_speculative_cycle_b200 import synth
+    cfg = synth.TINY
+    w = synth.make_drafter_weights(cfg, seed=seed, share_embed_lm_head=True)
+    feats = synth.make_features(cfg, P, seed=seed + 1)
+    cache = O.Cache(cfg)
+    cache.write(0, O.inject(cfg, w, feats, 0)[1])
+    return cfg, w, cache, feats
+
+
+def test_window_wider_than_the_context_is_no_window():
+    cfg, w, cache, _ = _window_case()
+    full = O.draft_block(cfg, w, 5, cache, 4)
+    for W in (40, 41, 1000):
+        win = O.draft_block(cfg, w, 5, cache, 4, window=W)
+        for a, b in zip(full["hidden"], win["hidden"]):
+            np.testing.assert_array_equal(a, b)
+
+
+def test_window_ignores_exactly_the_rows_before_it():
+    """Changing context rows older than the window leaves the pass unchanged; changing
+    the oldest row inside it does not."""
+    cfg, w, cache, feats = _window_case()
+    W, P = 16, 40
+    base = O.draft_block(cfg, w, 5, cache, 4, window=W)
+    old = O.Cache(cfg)
+    f2 = feats.clone()
+    f2[: P - W] = -f2[: P - W] * 3.0
+    old.write(0, O.inject(cfg, w, f2, 0)[1])
+    same = O.draft_block(cfg, w, 5, old, 4, window=W)
+    for a, b in zip(base["hidden"], same["hidden"]):
+        np.testing.assert_array_equal(a, b)
+    inside = O.Cache(cfg)
+    f3 = feats.clone()
+    f3[P - W] = -f3[P - W] * 3.0
+    inside.write(0, O.inject(cfg, w, f3, 0)[1])
+    moved = O.draft_block(cfg, w, 5, inside, 4, window=W)
+    assert np.abs(moved["hidden"][-1] - base["hidden"][-1]).max() > 1e-6
+
+
+def test_window_equals_a_cache_holding_only_its_rows():
+    """The window's rows keep their absolute positions: attending to the last W rows
+    of a long context is attending to a cache that holds only them, at the same P
+    (checked through the decoder library pin below: block_attention over the window
+    equals scaled_dot_product_attention over those keys)."""
+    import torch
+    cfg, w, cache, _ = _window_case()
+    W, P = 10, 40
+    win = O.draft_block(cfg, w, 7, cache, 4, window=W)
+    only = O.Cache.from_arrays(cfg, [k[P - W:P] for k in cache.k], [v[P - W:P] for v in cache.v])
+    ref = O.draft_block(cfg, w, 7, only, 4, ctx_len=P)   # positions P.., keys: the W kept rows
+    for a, b in zip(win["hidden"], ref["hidden"]):
+        np.testing.assert_array_equal(a, b)
+    # the first layer's attention of the windowed pass against SDPA on those keys
+    lw = w["layers"][0]
+    x = O.f64(w["embed"])[[7] + [cfg.mask_token_id] * 3]
+    h = O.rms_norm(x, lw["attn_norm"], cfg.rms_eps)
+    pos = np.arange(P, P + 4)
+    q = O.apply_rope(O.linear(h, lw["wq"]).reshape(4, cfg.n_q_heads, cfg.head_dim), pos, cfg.rope_theta)
+    k = O.apply_rope(O.linear(h, lw["wk"]).reshape(4, cfg.n_kv_heads, cfg.head_dim), pos, cfg.rope_theta)
+    v = O.linear(h, lw["wv"]).reshape(4, cfg.n_kv_heads, cfg.head_dim)
+    keys = np.concatenate([cache.k[0][P - W:P], k]); vals = np.concatenate([cache.v[0][P - W:P], v])
+    o = O.block_attention(q, keys, vals)
+    g = cfg.n_q_heads // cfg.n_kv_heads
+    tq = torch.from_numpy(q).permute(1, 0, 2)[None]
+    tk = torch.from_numpy(keys).permute(1, 0, 2).repeat_interleave(g, 0)[None]
+    tv = torch.from_numpy(vals).permute(1, 0, 2).repeat_interleave(g, 0)[None]
+    ref_o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)[0].permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(o, ref_o, rtol=1e-10, atol=1e-12)
