@@ -46,6 +46,9 @@ def parse_args():
     ap.add_argument("--profile-steps", type=int, default=10)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-budget-s", type=float, default=25.0)
+    ap.add_argument("--block-sweep", action="store_true",
+                    help="instead of the headline line: time the cycle at block sizes 4/8/10/16 at concurrency 1 "
+                         "and 32 and report the dynamic block-size policy's choice (one JSON line)")
     ap.add_argument("--kv-cache-dtype", default="f16", choices=["model", "f16"],
                     help="element type of the drafter's KV cache pools: f16 (bf16 drafters; same bytes as bf16, "
                          "3 more mantissa bits, read by the attention kernel without conversion) or the model dtype")
@@ -610,12 +613,90 @@ def stored_traffic(kernel: str, workload: str):
     return None
 
 
+def block_sweep(args, local):
+    """Dynamic block-size scheduling on measured cycles: for each concurrency, the
+    cycle (inject + draft + verify) is graph-timed at every candidate block size
+    with the same drafter, the acceptance lengths of those cycles (the planted
+    prefixes) feed the library's device acceptance counts, and the library's
+    policy picks the block with the most expected tokens per measured cycle time.
+    Prints one JSON line."""
+    import dataclasses
+    import torch
+    from block_diffusion_speculative_cycle_b200 import BlockPolicy, dflash_acceptance_count, dflash_verify, synth
+    cands, n_pos = [4, 8, 10, 16], 17
+    out = {"metric": "block-size policy on measured cycles", "candidates": cands, "rows": []}
+    dev = f"cuda:{local}"
+    for name in ("qwen8b_b16_serve_bs1", "qwen8b_b16_serve_bs32"):
+        w = synth.WORKLOADS[name]
+        c = Cycle(dataclasses.replace(w, block=max(cands)), dev, args.kv_cache_dtype)
+        counts = torch.zeros(2 * n_pos, dtype=torch.int64, device=dev)
+        row = {"workload": name, "batch": w.batch, "ms_per_cycle": {}, "expected_tokens": {}}
+        costs = []
+        for B in cands:
+            logits = c.logits[:, :B].contiguous()
+            draft = torch.zeros((c.bs, max(B - 1, 1)), dtype=torch.int32, device=dev)
+            n_new = torch.clamp(c.n_new, max=B).contiguous()
+            ws = torch.zeros(c.ws.numel(), dtype=torch.uint8, device=dev)
+
+            def cycle():
+                c.drafter.inject(c.feats, c.bs, c.B, n_new, c.start, c.kc, c.vc, c.table, c.num_pages)
+                c.drafter.draft(c.anchor, c.ctx, c.bs, B, c.kc, c.vc, c.table, c.num_pages, c.max_ctx, draft)
+                dflash_verify(logits, draft, c.acc, c.nxt, ws)
+            for _ in range(3):
+                cycle()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                cycle()
+            for _ in range(5):
+                g.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 30
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            row["ms_per_cycle"][B] = ms
+            costs.append(ms)
+            # The synthetic target accepts a geometric prefix (mean 6, the planted law) at
+            # any block size, clipped at B-1; the logits were planted against the
+            # block-16 draft, so a smaller block's own verify would mismatch for a
+            # synthetic reason. Clipped draws of that law feed the device counts.
+            # Acceptance statistics need many draws: 4096 seeded geometric lengths per block.
+            gen = torch.Generator().manual_seed(1234 + B)
+            p_geo = 1.0 / (1.0 + w.accept_mean)
+            u = torch.rand(4096, generator=gen, dtype=torch.float64)
+            geo = torch.floor(torch.log1p(-u) / math.log1p(-p_geo))
+            planted = torch.clamp(geo, max=B - 1).to(torch.int32).to(dev)
+            dflash_acceptance_count(planted, B, counts)
+            del g
+        torch.cuda.synchronize()
+        c.drafter.check()
+        cnt = counts.cpu().numpy()
+        pol = BlockPolicy(cands, 1.0, n_pos)
+        pol.observe(cnt[:n_pos], cnt[n_pos:])
+        for B in cands:
+            row["expected_tokens"][B] = pol.expected_tokens(B)
+        row["tokens_per_s"] = {B: c.bs * row["expected_tokens"][B] / (row["ms_per_cycle"][B] / 1e3) for B in cands}
+        row["policy_choice"] = pol.choose(costs)
+        row["best_by_measurement"] = max(cands, key=lambda B: row["tokens_per_s"][B])
+        out["rows"].append(row)
+        pol.close()
+        del c
+        torch.cuda.empty_cache()
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse_args()
     world, rank, local = setup_dist()
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.block_sweep:
+            block_sweep(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -24,7 +24,9 @@ _STATUS = {0: "DFLASH_OK", 1: "DFLASH_ERR_ARG", 2: "DFLASH_ERR_CUDA", 3: "DFLASH
 EXPORTS = ["dflash_create", "dflash_destroy", "dflash_inject_ctx", "dflash_draft_block", "dflash_draft_block_sample",
            "dflash_verify_sampled_workspace_size", "dflash_verify_sampled",
            "dflash_verify_workspace_size", "dflash_verify", "dflash_verify_noalloc", "dflash_profile_enable", "dflash_profile_read",
-           "dflash_profile_gemm_chain", "dflash_get_error", "dflash_status_string"]
+           "dflash_profile_gemm_chain", "dflash_get_error", "dflash_status_string", "dflash_acceptance_count",
+           "dflash_block_policy_create", "dflash_block_policy_destroy", "dflash_block_policy_observe",
+           "dflash_block_policy_expected_tokens", "dflash_block_policy_choose", "dflash_block_policy_choose_linear"]
 
 
 class DFlashError(RuntimeError):
@@ -98,6 +100,21 @@ def load_library(path: Optional[str] = None):
     lib.dflash_profile_read.restype = c_int
     lib.dflash_profile_gemm_chain.argtypes = [_P, _P, c_int, c_int, _P, _P, _PP, _PP, _P, c_int, c_int, _P, c_int, _P]
     lib.dflash_profile_gemm_chain.restype = c_int
+    c_dbl, c_u64p = ctypes.c_double, ctypes.POINTER(ctypes.c_ulonglong)
+    lib.dflash_acceptance_count.argtypes = [_P, c_int, c_int, _P, c_int, _P]
+    lib.dflash_acceptance_count.restype = c_int
+    lib.dflash_block_policy_create.argtypes = [ctypes.POINTER(c_int), c_int, c_dbl, c_int, ctypes.POINTER(_P)]
+    lib.dflash_block_policy_create.restype = c_int
+    lib.dflash_block_policy_destroy.argtypes = [_P]
+    lib.dflash_block_policy_destroy.restype = None
+    lib.dflash_block_policy_observe.argtypes = [_P, c_u64p, c_u64p, c_int]
+    lib.dflash_block_policy_observe.restype = c_int
+    lib.dflash_block_policy_expected_tokens.argtypes = [_P, c_int]
+    lib.dflash_block_policy_expected_tokens.restype = c_dbl
+    lib.dflash_block_policy_choose.argtypes = [_P, ctypes.POINTER(c_dbl), c_int]
+    lib.dflash_block_policy_choose.restype = c_int
+    lib.dflash_block_policy_choose_linear.argtypes = [_P, c_int, c_dbl, c_dbl]
+    lib.dflash_block_policy_choose_linear.restype = c_int
     lib.dflash_get_error.argtypes = [_P, _P]
     lib.dflash_get_error.restype = c_int
     lib.dflash_status_string.argtypes = [c_int]
@@ -246,6 +263,59 @@ def dflash_profile_gemm_chain(handle, feats, bs, max_new, n_new, start_pos, k_ca
                                          _ptr_array(k_cache), _ptr_array(v_cache), _ptr(page_table),
                                          page_table.shape[1], num_pages, _ptr(ctx_len), B, _stream(stream)),
            "dflash_profile_gemm_chain")
+
+
+def dflash_acceptance_count(accepted, B, counts, stream=None) -> None:
+    """counts: device uint64 (int64) tensor [2 * n_pos]: tested, then accepted per position."""
+    n_pos = counts.numel() // 2
+    _check(load_library().dflash_acceptance_count(_ptr(accepted), accepted.numel(), B, _ptr(counts), n_pos,
+                                                  _stream(stream)), "dflash_acceptance_count")
+
+
+class BlockPolicy:
+    """The library's block-size policy (host-side C++ object)."""
+
+    def __init__(self, candidates, decay: float, n_pos: int):
+        lib = load_library()
+        arr = (ctypes.c_int * len(candidates))(*[int(b) for b in candidates])
+        h = _P()
+        _check(lib.dflash_block_policy_create(arr, len(candidates), float(decay), n_pos, ctypes.byref(h)),
+               "dflash_block_policy_create")
+        self.handle, self.n_pos = h.value, n_pos
+        self.candidates = sorted(int(b) for b in candidates)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            load_library().dflash_block_policy_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def observe(self, tested, accepted) -> None:
+        t = (ctypes.c_ulonglong * self.n_pos)(*[int(x) for x in tested])
+        a = (ctypes.c_ulonglong * self.n_pos)(*[int(x) for x in accepted])
+        _check(load_library().dflash_block_policy_observe(self.handle, t, a, self.n_pos),
+               "dflash_block_policy_observe")
+
+    def expected_tokens(self, B: int) -> float:
+        return float(load_library().dflash_block_policy_expected_tokens(self.handle, B))
+
+    def choose(self, costs) -> int:
+        c = (ctypes.c_double * len(costs))(*[float(x) for x in costs])
+        r = load_library().dflash_block_policy_choose(self.handle, c, len(costs))
+        if r < 0:
+            raise DFlashError(-r, "dflash_block_policy_choose")
+        return r
+
+    def choose_linear(self, bs: int, c0: float, c1: float) -> int:
+        r = load_library().dflash_block_policy_choose_linear(self.handle, bs, float(c0), float(c1))
+        if r < 0:
+            raise DFlashError(-r, "dflash_block_policy_choose_linear")
+        return r
 
 
 def dflash_get_error(handle, stream=None) -> int:

@@ -269,6 +269,44 @@ dflash_status dflash_verify_sampled(const void* d_logits, dflash_dtype logits_dt
 dflash_status dflash_verify_noalloc(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft,
                                     int bs, int B, int V, int* d_accepted, int* d_next_token, void* stream);
 
+/* Dynamic block-size scheduling ([P3] §3 item 4 and §4: the drafter trained
+ * with block 16 also runs with smaller blocks, the block size scheduled
+ * dynamically). Reading taken: per-position acceptance rates
+ * alpha_i = P(draft i accepted | drafts 1..i-1 accepted), estimated from verify
+ * results with decayed counts and a Beta(1, 1) prior, alpha_i = (A_i + 1) / (T_i + 2);
+ * a cycle with block B commits 1 + sum_{i<B} prod_{j<=i} alpha_j tokens on
+ * average; the policy picks the candidate B with the most expected tokens per
+ * unit of the caller's cycle cost (the smaller B on an exact tie).
+ *
+ * dflash_acceptance_count: device side of the estimate. For each request r of a
+ * cycle run with block B (d_accepted [bs] int32, device, e.g. dflash_verify's
+ * output), adds 1 to d_counts[i] (tested) for positions 1 <= i <= min(a_r+1, B-1)
+ * and 1 to d_counts[n_pos + i] (accepted) for 1 <= i <= a_r. d_counts is a device
+ * array [2 * n_pos] of uint64 that the caller zero-fills and reads (integer
+ * atomics: exact and order-independent). B must not exceed n_pos. */
+dflash_status dflash_acceptance_count(const int* d_accepted, int bs, int B, unsigned long long* d_counts,
+                                      int n_pos, void* stream);
+
+/* Host-side policy (no GPU work). candidates: block sizes 1..n_pos to choose
+ * among; decay in (0, 1]: weight kept by past counts at each observation. */
+typedef struct dflash_block_policy dflash_block_policy;
+dflash_status dflash_block_policy_create(const int* candidates, int n_candidates, double decay, int n_pos,
+                                         dflash_block_policy** out);
+void dflash_block_policy_destroy(dflash_block_policy* policy);
+/* Fold one window of counts in (host copies of the two halves of d_counts above):
+ * T_i <- decay * T_i + tested[i], A_i <- decay * A_i + accepted[i]. */
+dflash_status dflash_block_policy_observe(dflash_block_policy* policy, const unsigned long long* tested,
+                                          const unsigned long long* accepted, int n_pos);
+/* Expected tokens committed by a cycle with block B (-1 for a B outside 1..n_pos). */
+double dflash_block_policy_expected_tokens(const dflash_block_policy* policy, int B);
+/* The candidate maximising expected tokens / costs[k] (costs in the candidates'
+ * ascending order, each > 0; e.g. measured cycle times at the current
+ * concurrency); a negative dflash_status on bad arguments. */
+int dflash_block_policy_choose(const dflash_block_policy* policy, const double* costs, int n_costs);
+/* The same with the cost model c0 + c1 * bs * B (c0: the cycle's fixed cost, c1:
+ * the cost of verifying one more token of one request). */
+int dflash_block_policy_choose_linear(const dflash_block_policy* policy, int bs, double c0, double c1);
+
 /* Per-kernel timing, an instrumentation hook with no counterpart on the pages.
  * While enabled, every kernel this context launches is bracketed by a pair of
  * CUDA events on its stream, tagged with the launch's algorithmic bytes (each
