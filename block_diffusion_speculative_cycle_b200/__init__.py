@@ -10,5 +10,6 @@ from ._binding import (  # noqa: F401
     dflash_get_error, dflash_inject_ctx, dflash_profile_enable, dflash_profile_gemm_chain, dflash_profile_read,
     dflash_status_string, dflash_verify, dflash_verify_workspace_size,
     dflash_draft_block_sample, dflash_verify_sampled, dflash_verify_sampled_workspace_size,
-    BlockPolicy, dflash_acceptance_count, exported_symbols, load_library, verify, verify_sampled,
+    BlockPolicy, dflash_acceptance_count, dflash_spec_commit, dflash_target_forward, exported_symbols, load_library,
+    verify, verify_sampled,
 )

@@ -26,7 +26,8 @@ EXPORTS = ["dflash_create", "dflash_destroy", "dflash_inject_ctx", "dflash_draft
            "dflash_verify_workspace_size", "dflash_verify", "dflash_verify_noalloc", "dflash_profile_enable", "dflash_profile_read",
            "dflash_profile_gemm_chain", "dflash_get_error", "dflash_status_string", "dflash_acceptance_count",
            "dflash_block_policy_create", "dflash_block_policy_destroy", "dflash_block_policy_observe",
-           "dflash_block_policy_expected_tokens", "dflash_block_policy_choose", "dflash_block_policy_choose_linear"]
+           "dflash_block_policy_expected_tokens", "dflash_block_policy_choose", "dflash_block_policy_choose_linear",
+           "dflash_target_forward", "dflash_spec_commit"]
 
 
 class DFlashError(RuntimeError):
@@ -115,6 +116,11 @@ def load_library(path: Optional[str] = None):
     lib.dflash_block_policy_choose.restype = c_int
     lib.dflash_block_policy_choose_linear.argtypes = [_P, c_int, c_dbl, c_dbl]
     lib.dflash_block_policy_choose_linear.restype = c_int
+    lib.dflash_target_forward.argtypes = [_P, _P, _P, _P, c_int, c_int, _P, _PP, _PP, _P, c_int, c_int, c_int,
+                                          ctypes.POINTER(c_int), c_int, _P, _P, _P]
+    lib.dflash_target_forward.restype = c_int
+    lib.dflash_spec_commit.argtypes = [c_int, c_int, _P, _P, _P, _P, c_int, _P, _P, _P, _P, _P, _P]
+    lib.dflash_spec_commit.restype = c_int
     lib.dflash_get_error.argtypes = [_P, _P]
     lib.dflash_get_error.restype = c_int
     lib.dflash_status_string.argtypes = [c_int]
@@ -316,6 +322,23 @@ class BlockPolicy:
         if r < 0:
             raise DFlashError(-r, "dflash_block_policy_choose_linear")
         return r
+
+
+def dflash_target_forward(handle, tokens, anchor, draft, bs, n, pos0, k_cache, v_cache, page_table, num_pages,
+                          max_ctx, taps, logits, feats, stream=None) -> None:
+    lib = load_library()
+    tp = (ctypes.c_int * max(1, len(taps)))(*[int(t) for t in taps])
+    _check(lib.dflash_target_forward(handle, _ptr(tokens), _ptr(anchor), _ptr(draft), bs, n, _ptr(pos0),
+                                     _ptr_array(k_cache), _ptr_array(v_cache), _ptr(page_table), page_table.shape[1],
+                                     num_pages, max_ctx, tp, len(taps), _ptr(logits), _ptr(feats), _stream(stream)),
+           "dflash_target_forward")
+
+
+def dflash_spec_commit(bs, B, draft, accepted, next_token, out_tokens, out_len, anchor, ctx_len, n_new, start_pos,
+                       stream=None) -> None:
+    _check(load_library().dflash_spec_commit(bs, B, _ptr(draft), _ptr(accepted), _ptr(next_token), _ptr(out_tokens),
+                                              out_tokens.shape[1], _ptr(out_len), _ptr(anchor), _ptr(ctx_len),
+                                              _ptr(n_new), _ptr(start_pos), _stream(stream)), "dflash_spec_commit")
 
 
 def dflash_get_error(handle, stream=None) -> int:

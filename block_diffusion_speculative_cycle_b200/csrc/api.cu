@@ -828,7 +828,8 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
     const double es = (double)esize(ctx);
     {
       ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
-      DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, B, R, c.vocab, H,
+      DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, nullptr, nullptr, B, R,
+                                              c.vocab, H,
                                               c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps,
                                               ctx->x, ctx->h, hb, hb ? (size_t)R * H : 0, ctx->status, st,
                                               ctx->use_pdl),
@@ -1128,4 +1129,115 @@ extern "C" dflash_status dflash_profile_gemm_chain(dflash_ctx* ctx, const void* 
   } catch (...) {   // no C++ exception crosses the C ABI
     return DFLASH_ERR_OOM;
   }
+}
+
+extern "C" dflash_status dflash_target_forward(dflash_ctx* ctx, const int* d_tokens, const int* d_anchor,
+                                               const int* d_draft, int bs, int n, const int* d_pos0,
+                                               void* const* k_cache, void* const* v_cache, const int* d_page_table,
+                                               int max_pages, int num_pages, int max_ctx, const int* taps, int n_taps,
+                                               float* d_logits, float* d_feats, void* stream) {
+  dfl::TraceRange trace_("dflash_target_forward");
+  try {
+    if (!ctx) return DFLASH_ERR_ARG;
+    const dflash_config& c = ctx->cfg;
+    if (ctx->bf16) return DFLASH_ERR_UNSUPPORTED;   // the causal path is the fp32 one
+    if (bs <= 0 || bs > c.max_batch || n <= 0 || n > c.max_block || max_ctx < 0) return DFLASH_ERR_ARG;
+    if (!d_tokens && (!d_anchor || (n > 1 && !d_draft))) return DFLASH_ERR_ARG;
+    if (!d_pos0 || !d_page_table || max_pages <= 0 || num_pages <= 0 || !d_logits) return DFLASH_ERR_ARG;
+    if (c.n_layers > 0 && (!k_cache || !v_cache)) return DFLASH_ERR_ARG;
+    for (int l = 0; l < c.n_layers; ++l)
+      if (!k_cache[l] || !v_cache[l]) return DFLASH_ERR_ARG;
+    if (n_taps < 0 || (n_taps > 0 && (!taps || !d_feats))) return DFLASH_ERR_ARG;
+    for (int f = 0; f < n_taps; ++f)
+      if (taps[f] < 0 || taps[f] >= c.n_layers || (f > 0 && taps[f] <= taps[f - 1])) return DFLASH_ERR_ARG;
+    if ((long long)max_ctx + n > (long long)max_pages * c.page_size) return DFLASH_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int R = bs * n;
+    const int H = c.hidden, KVD = kv_dim(c);
+
+    DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, 0, d_anchor, c.mask_token_id, d_tokens, d_draft, n, R,
+                                            c.vocab, H, c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm,
+                                            c.rms_eps, ctx->x, ctx->h, 0, 0, ctx->status, st, ctx->use_pdl),
+                          "embed_norm launch"));
+    // The split plan depends on bs and max_ctx only (not on n or the rows' positions),
+    // so a row's attention is the same arithmetic in a block forward and in a
+    // one-token forward given the same max_ctx.
+    const int g = c.n_q_heads / c.n_kv_heads;
+    const int pairs = bs * c.n_kv_heads;
+    int n_splits = std::max(1, (kAttnTargetCtas + pairs - 1) / pairs);
+    int kps = (std::max(max_ctx, 1) + n_splits - 1) / n_splits;
+    kps = (kps + 31) / 32 * 32;
+    n_splits = std::max(1, (max_ctx + kps - 1) / kps);
+    if ((size_t)bs * c.n_kv_heads * n_splits * g * n > ctx->att_rows) return DFLASH_ERR_UNSUPPORTED;
+
+    for (int l = 0; l < c.n_layers; ++l) {
+      DFL_CHECK(run_gemm(ctx, spec_qkv(ctx, l, R, n, d_pos0), st));
+      // the block's own keys and values join the target's cache (a causal decoder)
+      DFL_CHECK(cuda_status(launch_kv_scatter((const float*)ctx->kb, (const float*)ctx->vb, d_pos0, n, R, c.n_kv_heads,
+                                              c.head_dim, d_page_table, max_pages, num_pages, c.page_size,
+                                              (float*)k_cache[l], (float*)v_cache[l], ctx->status, st),
+                            "kv scatter launch"));
+      AttnParams ap{};
+      ap.q = ctx->q;
+      ap.kblk = ctx->kb;
+      ap.vblk = ctx->vb;
+      ap.kc = k_cache[l];
+      ap.vc = v_cache[l];
+      ap.ctx_len = d_pos0;   // context: cache positions before the block
+      ap.page_table = d_page_table;
+      ap.max_pages = max_pages;
+      ap.num_pages = num_pages;
+      ap.page_size = c.page_size;
+      ap.bs = bs;
+      ap.B = n;
+      ap.n_q = c.n_q_heads;
+      ap.n_kv = c.n_kv_heads;
+      ap.d = c.head_dim;
+      ap.g = g;
+      ap.kps = kps;
+      ap.n_splits = n_splits;
+      ap.ks = 1;
+      ap.max_ctx = max_ctx;
+      ap.scale = (float)(1.0 / std::sqrt((double)c.head_dim));
+      ap.part_o = ctx->att_o;
+      ap.part_m = ctx->att_m;
+      ap.part_l = ctx->att_l;
+      ap.status = ctx->status;
+      ap.causal = 1;
+      DFL_CHECK(cuda_status(launch_attention(ap, ctx->ao, 0, 0, st, ctx->use_pdl), "attention launch"));
+      DFL_CHECK(run_gemm(ctx, spec_o(ctx, l, R), st));
+      DFL_CHECK(run_gemm(ctx, spec_gateup(ctx, l, R), st));
+      DFL_CHECK(run_gemm(ctx, spec_down(ctx, l, R), st));
+      for (int f = 0; f < n_taps; ++f)
+        if (taps[f] == l && cudaMemcpy2DAsync(d_feats + (size_t)f * H, (size_t)n_taps * H * 4, ctx->x, (size_t)H * 4,
+                                              (size_t)H * 4, (size_t)R, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+          return DFLASH_ERR_CUDA;
+    }
+    // final norm (deferred) -> LM head, every row's logits stored
+    GemmSpec lm = spec_lm(ctx, R);
+    lm.epi.kind = EPI_STORE;
+    lm.epi.out[0] = d_logits;
+    lm.epi.ld_out[0] = c.vocab;
+    lm.epi.rows_per_req = n;
+    if (c.n_layers == 0)
+      DFL_CHECK(cuda_status(launch_rmsnorm(ctx->x, R, H, ctx->final_norm, c.rms_eps, ctx->h, 0, nullptr, st,
+                                           ctx->use_pdl),
+                            "rmsnorm launch"));
+    return run_gemm(ctx, lm, st);
+  } catch (...) {   // no C++ exception crosses the C ABI
+    return DFLASH_ERR_OOM;
+  }
+}
+
+extern "C" dflash_status dflash_spec_commit(int bs, int B, const int* d_draft, const int* d_accepted,
+                                            const int* d_next_token, int* d_out_tokens, int max_out, int* d_out_len,
+                                            int* d_anchor, int* d_ctx_len, int* d_n_new, int* d_start_pos,
+                                            void* stream) {
+  if (bs <= 0 || B <= 0 || max_out <= 0 || (B > 1 && !d_draft) || !d_accepted || !d_next_token || !d_out_tokens ||
+      !d_out_len || !d_anchor || !d_ctx_len || !d_n_new || !d_start_pos)
+    return DFLASH_ERR_ARG;
+  return cuda_status(launch_spec_commit(bs, B, d_draft, d_accepted, d_next_token, d_out_tokens, max_out, d_out_len,
+                                        d_anchor, d_ctx_len, d_n_new, d_start_pos,
+                                        reinterpret_cast<cudaStream_t>(stream)),
+                     "spec commit launch");
 }

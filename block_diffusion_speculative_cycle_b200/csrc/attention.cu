@@ -85,14 +85,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_kernel(const AttnPara
       const int r = warp + 8 * rr;
       if (r < nr) {
         float sc = -INFINITY;
-        if (valid) {
+        // a causal decoder's row i (position P + i) sees block keys 0..i only
+        if (valid && !(p.causal && kt + lane >= P && kt + lane - P > r % p.B)) {
           float dot = 0.f;
 #pragma unroll 8
           for (int dd = 0; dd < D; ++dd) dot = fmaf(qs[r * D + dd], ks[lane * (D + 1) + dd], dot);
           sc = dot;
         }
         const float mn = fmaxf(m[rr], warp_max(sc));
-        const float pe = valid ? expf(sc - mn) : 0.f;
+        const float pe = sc != -INFINITY ? expf(sc - mn) : 0.f;
         // a tile with every key masked (below a sliding window's start) while the
         // row has seen no key yet leaves the state as it is
         const float alpha = mn == -INFINITY ? 1.f : expf(m[rr] - mn);

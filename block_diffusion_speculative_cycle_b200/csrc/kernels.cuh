@@ -28,6 +28,7 @@ struct AttnParams {
   int cache_f16;              // tensor-core path: the cache pools hold fp16 (else bf16, converted on load)
   int global_merge;           // tensor-core path: splits write part_o/m/l (exp2 domain) and a second kernel merges
   int window;                 // sliding window: the block sees context positions P-window .. P-1 only (0: all)
+  int causal;                 // fp32 path only: block row i sees block keys 0..i (a causal decoder), not all B
 };
 
 // First context key the block attends to, and the 64-aligned key where split 0
@@ -71,14 +72,26 @@ int attn_tc_max_clusters(int d, bool compact, int stages, int n, bool gmerge, in
 // CUDA-core split-KV attention partials (fp32 path), then the log-sum-exp merge into out [R, n_q*d].
 cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int in_bf16, cudaStream_t st, bool pdl);
 
-// x[m] = E[token(m)] (token = anchor for block index 0, mask id otherwise), h[m] = RMSNorm(x[m]) * gain.
+// x[m] = E[token(m)], h[m] = RMSNorm(x[m]) * gain. token(m) for row m (request m / B,
+// position i = m % B): tokens[m] when tokens is given; else the anchor at i = 0 and
+// draft[request, i-1] (when draft is given) or the mask id at i >= 1.
 // With h_plane != 0 (bf16 h), h is written as hi/lo planes h_plane elements apart.
-cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
-                              int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
+cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, const int* tokens,
+                              const int* draft, int B, int R, int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
                               int* status, cudaStream_t st, bool pdl);
 // h[m] = RMSNorm(x[m]) * gain into h (model dtype) and/or y (fp32); either may be null.
 cudaError_t launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
                            cudaStream_t st, bool pdl);
+// Copy the block's k / v rows (fp32 [R, n_kv*d], row m = request m / n, position
+// pos0[request] + m % n) into the page pools [num_pages, n_kv, page_size, d];
+// rows whose page slot or page id is out of range are skipped and flagged.
+cudaError_t launch_kv_scatter(const float* kb, const float* vb, const int* pos0, int n, int R, int n_kv, int d,
+                              const int* page_table, int max_pages, int num_pages, int page_size, float* kc, float* vc,
+                              int* status, cudaStream_t st);
+// Device-side commit of one speculative cycle per request (see dflash_spec_commit).
+cudaError_t launch_spec_commit(int bs, int B, const int* draft, const int* accepted, const int* next_token,
+                               int* out_tokens, int max_out, int* out_len, int* anchor, int* ctx_len, int* n_new,
+                               int* start_pos, cudaStream_t st);
 // draft[b, i-1] = index(keys[b*B + i]) for i >= 1; every key reset to 0.
 cudaError_t launch_argmax_finalize(unsigned long long* keys, int bs, int B, int* draft, cudaStream_t st, bool pdl);
 

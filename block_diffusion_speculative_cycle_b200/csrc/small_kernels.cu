@@ -77,14 +77,17 @@ __device__ __forceinline__ void norm_store(const float4* v, float ss, int H, con
 
 template <int VPT, typename ET, typename HT>
 __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const ET* embed, const int* anchor, int mask_id,
-                                                                  int B, int V, int H, const float* gain,
-                                                                  float eps, float* x, HT* h, size_t h_plane,
-                                                                  int* status) {
+                                                                  const int* tokens, const int* draft, int B, int V,
+                                                                  int H, const float* gain, float eps, float* x, HT* h,
+                                                                  size_t h_plane, int* status) {
   __shared__ float red[32];
   grid_dep_wait();
   grid_dep_launch();
   const int m = blockIdx.x;
-  int tok = (m % B) == 0 ? anchor[m / B] : mask_id;
+  // row (request m / B, position m % B): tokens[m] when given; else the anchor at
+  // position 0 and, at positions i >= 1, draft[request, i-1] (given) or the mask id
+  const int i = m % B;
+  int tok = tokens ? tokens[m] : (i == 0 ? anchor[m / B] : (draft ? draft[(size_t)(m / B) * (B - 1) + i - 1] : mask_id));
   if (tok < 0 || tok >= V) {
     if (threadIdx.x == 0) flag_error(status, ST_BAD_TOKEN);
     tok = 0;
@@ -133,39 +136,39 @@ __global__ void argmax_finalize_kernel(unsigned long long* keys, int bs, int B, 
 }
 
 template <int VPT>
-static cudaError_t embed_norm_vpt(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R,
-                                  int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16,
+static cudaError_t embed_norm_vpt(const void* embed, int embed_bf16, const int* anchor, int mask_id,
+                                  const int* tokens, const int* draft, int B, int R, int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16,
                                   size_t h_plane, int* status, cudaStream_t st, bool pdl) {
   const dim3 g(R), b(kNormThreads);
   if (embed_bf16 && h_bf16)
     return launch_kernel(embed_norm_kernel<VPT, __nv_bfloat16, __nv_bfloat16>, g, b, 0, st, pdl,
-                         (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h,
+                         (const __nv_bfloat16*)embed, anchor, mask_id, tokens, draft, B, V, H, gain, eps, x, (__nv_bfloat16*)h,
                          h_plane, status);
   if (!embed_bf16 && !h_bf16)
     return launch_kernel(embed_norm_kernel<VPT, float, float>, g, b, 0, st, pdl, (const float*)embed, anchor,
-                         mask_id, B, V, H, gain, eps, x, (float*)h, (size_t)0, status);
+                         mask_id, tokens, draft, B, V, H, gain, eps, x, (float*)h, (size_t)0, status);
   if (embed_bf16)
     return launch_kernel(embed_norm_kernel<VPT, __nv_bfloat16, float>, g, b, 0, st, pdl,
-                         (const __nv_bfloat16*)embed, anchor, mask_id, B, V, H, gain, eps, x, (float*)h, (size_t)0,
+                         (const __nv_bfloat16*)embed, anchor, mask_id, tokens, draft, B, V, H, gain, eps, x, (float*)h, (size_t)0,
                          status);
   return launch_kernel(embed_norm_kernel<VPT, float, __nv_bfloat16>, g, b, 0, st, pdl, (const float*)embed, anchor,
-                       mask_id, B, V, H, gain, eps, x, (__nv_bfloat16*)h, h_plane, status);
+                       mask_id, tokens, draft, B, V, H, gain, eps, x, (__nv_bfloat16*)h, h_plane, status);
 }
 
-cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, int B, int R, int V,
-                              int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
+cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, const int* tokens,
+                              const int* draft, int B, int R, int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
                               int* status, cudaStream_t st, bool pdl) {
   const int vpt = (H / 4 + kNormThreads - 1) / kNormThreads;
   if (vpt <= 1)
-    return embed_norm_vpt<1>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
+    return embed_norm_vpt<1>(embed, embed_bf16, anchor, mask_id, tokens, draft, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
                              st, pdl);
   if (vpt <= 2)
-    return embed_norm_vpt<2>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
+    return embed_norm_vpt<2>(embed, embed_bf16, anchor, mask_id, tokens, draft, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
                              st, pdl);
   if (vpt <= 4)
-    return embed_norm_vpt<4>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
+    return embed_norm_vpt<4>(embed, embed_bf16, anchor, mask_id, tokens, draft, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
                              st, pdl);
-  return embed_norm_vpt<8>(embed, embed_bf16, anchor, mask_id, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
+  return embed_norm_vpt<8>(embed, embed_bf16, anchor, mask_id, tokens, draft, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
                            st, pdl);
 }
 
@@ -191,6 +194,72 @@ cudaError_t launch_rmsnorm(const float* x, int R, int H, const float* gain, floa
 cudaError_t launch_argmax_finalize(unsigned long long* keys, int bs, int B, int* draft, cudaStream_t st, bool pdl) {
   const int n = bs * B;
   return launch_kernel(argmax_finalize_kernel, dim3((n + 255) / 256), dim3(256), 0, st, pdl, keys, bs, B, draft);
+}
+
+}  // namespace dfl
+
+namespace dfl {
+
+// One block per row: copy the row's n_kv*d keys and values into its cache page.
+__global__ void __launch_bounds__(128) kv_scatter_kernel(const float* kb, const float* vb, const int* pos0, int n,
+                                                         int n_kv, int d, const int* page_table, int max_pages,
+                                                         int num_pages, int page_size, float* kc, float* vc,
+                                                         int* status) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int m = blockIdx.x;
+  const int req = m / n;
+  const int pos = pos0[req] + m % n;
+  const int slot = pos >= 0 ? pos / page_size : -1;
+  const int page = slot >= 0 && slot < max_pages ? page_table[(size_t)req * max_pages + slot] : -1;
+  if (page < 0 || page >= num_pages) {
+    if (threadIdx.x == 0) flag_error(status, ST_BAD_PAGE);
+    return;
+  }
+  const int kvd = n_kv * d;
+  for (int e = threadIdx.x; e < kvd; e += blockDim.x) {
+    const int head = e / d, j = e % d;
+    const size_t dst = (((size_t)page * n_kv + head) * page_size + pos % page_size) * d + j;
+    kc[dst] = kb[(size_t)m * kvd + e];
+    vc[dst] = vb[(size_t)m * kvd + e];
+  }
+}
+
+cudaError_t launch_kv_scatter(const float* kb, const float* vb, const int* pos0, int n, int R, int n_kv, int d,
+                              const int* page_table, int max_pages, int num_pages, int page_size, float* kc, float* vc,
+                              int* status, cudaStream_t st) {
+  return launch_kernel(kv_scatter_kernel, dim3(R), dim3(128), 0, st, true, kb, vb, pos0, n, n_kv, d, page_table,
+                       max_pages, num_pages, page_size, kc, vc, status);
+}
+
+// One thread per request: commit d_1..d_a and next, then advance the request's
+// state for the next cycle (anchor, context length, injection rows and start).
+__global__ void spec_commit_kernel(int bs, int B, const int* draft, const int* accepted, const int* next_token,
+                                   int* out_tokens, int max_out, int* out_len, int* anchor, int* ctx_len, int* n_new,
+                                   int* start_pos) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= bs) return;
+  const int a = accepted[b], nxt = next_token[b];
+  int len = out_len[b];
+  int* out = out_tokens + (size_t)b * max_out;
+  for (int i = 0; i < a; ++i)
+    if (len < max_out) out[len++] = draft[(size_t)b * (B - 1) + i];
+  if (len < max_out) out[len++] = nxt;
+  out_len[b] = len;
+  const int P = ctx_len[b];
+  start_pos[b] = P;
+  n_new[b] = a + 1;
+  ctx_len[b] = P + a + 1;
+  anchor[b] = nxt;
+}
+
+cudaError_t launch_spec_commit(int bs, int B, const int* draft, const int* accepted, const int* next_token,
+                               int* out_tokens, int max_out, int* out_len, int* anchor, int* ctx_len, int* n_new,
+                               int* start_pos, cudaStream_t st) {
+  return launch_kernel(spec_commit_kernel, dim3((bs + 127) / 128), dim3(128), 0, st, true, bs, B, draft, accepted,
+                       next_token, out_tokens, max_out, out_len, anchor, ctx_len, n_new, start_pos);
 }
 
 }  // namespace dfl

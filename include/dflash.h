@@ -269,6 +269,45 @@ dflash_status dflash_verify_sampled(const void* d_logits, dflash_dtype logits_dt
 dflash_status dflash_verify_noalloc(const void* d_logits, dflash_dtype logits_dtype, const int* d_draft,
                                     int bs, int B, int V, int* d_accepted, int* d_next_token, void* stream);
 
+/* A causal target forward for the speculative loop on the device ([P4] "DFlash
+ * 소개": spec_generate(target, draft, ...); [P1] §1-2: the target verifies the
+ * block in one forward pass and its features feed the drafter). The context must
+ * come from dflash_create with the TARGET's weights, fp32 (DFLASH_ERR_UNSUPPORTED
+ * for bf16); `fc` and the feature fields are not used. It runs the same layer
+ * (pre-norm RMSNorm, GQA with RoPE, SwiGLU) causally over n rows per request:
+ * row i of request r is position pos0[r] + i and attends to the target cache's
+ * positions < pos0[r] and to rows 0..i; its own K/V are written into the cache
+ * (so rows past the accepted ones are simply overwritten later: truncation is
+ * the caller's context length). No sliding window.
+ *   d_tokens   [bs, n] int32, or NULL: row 0 = d_anchor[r], row i = d_draft[r, i-1]
+ *              (the verify block [anchor, d_1 .. d_{n-1}])
+ *   d_pos0     [bs] int32 (device): position of each request's row 0
+ *   k_cache, v_cache, d_page_table, max_pages, num_pages: the target's own page
+ *              pools and table (layout as for dflash_inject_ctx)
+ *   max_ctx    host bound on every pos0: the attention split plan depends on bs and
+ *              max_ctx only, so with the same max_ctx a row's logits are the same
+ *              bits in a block forward and in a one-row forward
+ *   taps       HOST array of n_taps ascending layer indices; d_feats [bs, n, n_taps*H]
+ *              fp32 (out) receives the residual stream after each tapped layer,
+ *              concatenated shallow to deep (the drafter's injection features)
+ *   d_logits   [bs, n, V] fp32 (out) */
+dflash_status dflash_target_forward(dflash_ctx* ctx, const int* d_tokens, const int* d_anchor, const int* d_draft,
+                                    int bs, int n, const int* d_pos0, void* const* k_cache, void* const* v_cache,
+                                    const int* d_page_table, int max_pages, int num_pages, int max_ctx,
+                                    const int* taps, int n_taps, float* d_logits, float* d_feats, void* stream);
+
+/* Device-side control of the speculative loop ([P1] §2 steps 1-4 and §1: the
+ * accepted drafts and the correction are committed). Per request r, after
+ * dflash_verify gave (a, next) for the block drafted at context length P = ctx_len[r]:
+ * appends draft[r, 0..a-1] and next to out_tokens[r, out_len[r] ..] (at most
+ * max_out tokens per request), then sets start_pos[r] = P, n_new[r] = a + 1 (the
+ * committed block rows whose target features are injected next), ctx_len[r] = P + a + 1
+ * and anchor[r] = next. All arrays are device int32 [bs] ([bs, max_out] for
+ * out_tokens, [bs, B-1] for draft); nothing is read back to the host. */
+dflash_status dflash_spec_commit(int bs, int B, const int* d_draft, const int* d_accepted, const int* d_next_token,
+                                 int* d_out_tokens, int max_out, int* d_out_len, int* d_anchor, int* d_ctx_len,
+                                 int* d_n_new, int* d_start_pos, void* stream);
+
 /* Dynamic block-size scheduling ([P3] §3 item 4 and §4: the drafter trained
  * with block 16 also runs with smaller blocks, the block size scheduled
  * dynamically). Reading taken: per-position acceptance rates
