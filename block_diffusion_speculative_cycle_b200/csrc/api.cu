@@ -68,6 +68,10 @@ struct dflash_ctx {
   int attn_form = -1;           // DFLASH_ATTN_FORM=full|compact: force the tcgen05 attention form (experiments)
   int attn_l2promo = 3;         // DFLASH_ATTN_L2PROMO=0..3: L2 promotion of the attention's tensor maps (experiments)
   int attn_stages = 5;          // K/V ring depth of the tcgen05 attention (DFLASH_ATTN_STAGES, experiments)
+  // GEMM sites (bit 1 kv, 2 qkv, 3 o, 4 gate/up, 5 down) that read their activations
+  // as one bf16 plane from single_plane_rows rows on (DFLASH_SINGLE_PLANE=mask,rows)
+  unsigned single_plane_mask = 0;
+  int single_plane_rows = 1 << 30;
   std::map<std::tuple<int, int, int, int>, int> attn_cluster_cap;   // resident clusters per (d, stages, n, rows)
   int num_sms = 148;
   const void* fc = nullptr;
@@ -209,6 +213,14 @@ struct GemmSpec {
   EpiParams epi{};
 };
 
+enum { SITE_KV = 1, SITE_QKV = 2, SITE_O = 3, SITE_GATEUP = 4, SITE_DOWN = 5 };
+
+// Whether a GEMM site reads its activations as hi/lo planes at `rows` rows.
+bool two_planes(const dflash_ctx* ctx, int site, int rows) {
+  if (!ctx->bf16) return false;
+  return !((ctx->single_plane_mask >> site) & 1u) || rows < ctx->single_plane_rows;
+}
+
 // K splits per output tile (= cluster size): the largest count (<= 8) that keeps
 // the grid within split_slots CTAs per SM (default two), so every CTA streams
 // from the start and a third slot per SM stays free for the next kernel's CTAs
@@ -342,7 +354,7 @@ GemmSpec spec_qkv(dflash_ctx* ctx, int l, int R, int B, const int* d_ctx_len) {
   const int QD = q_dim(c), KVD = kv_dim(c);
   GemmSpec qkv;
   qkv.x = ctx->h;
-  qkv.x_split = ctx->bf16;
+  qkv.x_split = two_planes(ctx, SITE_QKV, R);
   qkv.ldx = c.hidden;
   qkv.M = R;
   qkv.K = c.hidden;
@@ -376,7 +388,7 @@ GemmSpec spec_o(dflash_ctx* ctx, int l, int R) {
   const dflash_config& c = ctx->cfg;
   GemmSpec o;
   o.x = ctx->ao;
-  o.x_split = ctx->bf16;
+  o.x_split = two_planes(ctx, SITE_O, R);
   o.ldx = q_dim(c);
   o.M = R;
   o.K = q_dim(c);
@@ -401,7 +413,7 @@ GemmSpec spec_gateup(dflash_ctx* ctx, int l, int R) {
   const dflash_config& c = ctx->cfg;
   GemmSpec gu;
   gu.x = ctx->h;
-  gu.x_split = ctx->bf16;
+  gu.x_split = two_planes(ctx, SITE_GATEUP, R);
   gu.ldx = c.hidden;
   gu.M = R;
   gu.K = c.hidden;
@@ -425,7 +437,7 @@ GemmSpec spec_down(dflash_ctx* ctx, int l, int R) {
   const dflash_config& c = ctx->cfg;
   GemmSpec dn;
   dn.x = ctx->act;
-  dn.x_split = ctx->bf16;
+  dn.x_split = two_planes(ctx, SITE_DOWN, R);
   dn.ldx = c.intermediate;
   dn.M = R;
   dn.K = c.intermediate;
@@ -542,6 +554,15 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     if (env) ctx->attn_form = std::strcmp(env, "compact") == 0 ? 1 : (std::strcmp(env, "full") == 0 ? 0 : -1);
     env = std::getenv("DFLASH_ATTN_L2PROMO");
     if (env && std::atoi(env) >= 0 && std::atoi(env) <= 3) ctx->attn_l2promo = std::atoi(env);
+    env = std::getenv("DFLASH_SINGLE_PLANE");
+    if (env) {
+      unsigned mask = 0;
+      int rows = 0;
+      if (std::sscanf(env, "%u,%d", &mask, &rows) == 2 && rows >= 0) {
+        ctx->single_plane_mask = mask;
+        ctx->single_plane_rows = rows;
+      }
+    }
     env = std::getenv("DFLASH_ATTN_STAGES");
     if (env && std::atoi(env) >= 2 && std::atoi(env) <= kMaxAttnTcStages) ctx->attn_stages = std::atoi(env);
     if (c.head_dim == 128 && ctx->attn_stages > 5) ctx->attn_stages = 5;   // what fits beside Q and P
@@ -761,7 +782,7 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
       const int nl = std::min(per_launch, c.n_layers - l0);
       GemmSpec kv;
       kv.x = ctx->c;
-      kv.x_split = ctx->bf16;
+      kv.x_split = two_planes(ctx, SITE_KV, M);
       kv.ldx = c.hidden;
       kv.M = M;
       kv.K = c.hidden;

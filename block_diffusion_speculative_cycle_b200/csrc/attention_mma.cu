@@ -555,17 +555,20 @@ static size_t attn_cluster_smem(int d, int nr, int rows_pad, int nst, int ks, in
   return loads > merge ? loads : merge;
 }
 
-// Global merge (many splits): one warp per (block row, query head) combines the
-// splits that hold keys (log-sum-exp weights in the exp2 domain, split order)
-// and writes the row as bf16 hi/lo planes.
+// Global merge (many splits): one CTA per (block row, query head). Its four warps
+// take the splits that hold keys in turn (split s to warp s % 4), each lane a
+// contiguous run of D/32 output columns, so every warp has its loads in flight
+// together; the warps' sums meet in shared memory. Log-sum-exp weights in the
+// exp2 domain; the row is written as bf16 hi/lo planes.
 template <int D>
-__global__ void __launch_bounds__(256) attn_gmerge_kernel(const AttnParams p, __nv_bfloat16* out) {
+__global__ void __launch_bounds__(128) attn_gmerge_kernel(const AttnParams p, __nv_bfloat16* out) {
+  constexpr int DPL = D / 32;   // columns per lane: 4 (D = 128) or 2 (D = 64)
+  __shared__ float red_m[4], red_l[4];
+  __shared__ __align__(16) float red_o[4][D];
   grid_dep_wait();
   grid_dep_launch();
-  const int gw = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  const int R = p.bs * p.B;
-  if (gw >= R * p.n_q) return;
-  const int m_row = gw / p.n_q, j = gw % p.n_q;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_row = blockIdx.x / p.n_q, j = blockIdx.x % p.n_q;
   const int b = m_row / p.B, i = m_row % p.B;
   const int h = j / p.g, jj = j % p.g;
   const int nr = p.g * p.B, r = jj * p.B + i;
@@ -573,53 +576,57 @@ __global__ void __launch_bounds__(256) attn_gmerge_kernel(const AttnParams p, __
   P = P < 0 ? 0 : (P > p.max_ctx ? p.max_ctx : P);
   const int used = min(p.n_splits, (P + p.B - attn_key_base(attn_ctx_lo(P, p.window)) + p.kps - 1) / p.kps);
   const size_t base = (size_t)(b * p.n_kv + h) * p.n_splits * nr + r;
+  // the row's maximum over the splits
   float M = -INFINITY;
-  for (int s = lane; s < used; s += 32) M = fmaxf(M, __ldcg(p.part_m + base + (size_t)s * nr));
+  for (int s = threadIdx.x; s < used; s += 128) M = fmaxf(M, __ldcg(p.part_m + base + (size_t)s * nr));
   M = warp_max(M);
-  float L = 0.f;
-  for (int s = lane; s < used; s += 32) {
+  if (lane == 0) red_m[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+  // this warp's splits: sum of 2^(m_s - M) * (l_s, o_s)
+  float acc[DPL], L = 0.f;
+#pragma unroll
+  for (int c = 0; c < DPL; ++c) acc[c] = 0.f;
+#pragma unroll 4
+  for (int s = warp; s < used; s += 4) {
     const size_t idx = base + (size_t)s * nr;
     const float ms = __ldcg(p.part_m + idx);
-    L += ms == -INFINITY ? 0.f : __ldcg(p.part_l + idx) * exp2f(ms - M);
-  }
-  L = warp_sum(L);
-  const float invL = 1.f / L;
-  float acc[D / 32];
-#pragma unroll
-  for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
-  for (int s0 = 0; s0 < used; s0 += 32) {
-    const int sl = s0 + lane;
-    float wl = 0.f;
-    if (sl < used) {
-      const float ms = __ldcg(p.part_m + base + (size_t)sl * nr);
-      wl = ms == -INFINITY ? 0.f : exp2f(ms - M) * invL;
-    }
-    const int n = min(32, used - s0);
-#pragma unroll 4
-    for (int k = 0; k < n; ++k) {
-      const float w = __shfl_sync(0xffffffffu, wl, k);
-      const float* o = p.part_o + (base + (size_t)(s0 + k) * nr) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) acc[c] = fmaf(w, __ldcg(o + lane + 32 * c), acc[c]);
+    const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
+    L = fmaf(w, __ldcg(p.part_l + idx), L);
+    const float* o = p.part_o + idx * D + lane * DPL;
+    if constexpr (DPL == 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(o));
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+      acc[2] = fmaf(w, v.z, acc[2]);
+      acc[3] = fmaf(w, v.w, acc[3]);
+    } else {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(o));
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
     }
   }
-  __nv_bfloat16* dst = out + (size_t)m_row * p.n_q * D + j * D;
+  if (lane == 0) red_l[warp] = L;
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
-    const __nv_bfloat16 hi = __float2bfloat16_rn(acc[c]);
-    dst[lane + 32 * c] = hi;
-    dst[lane + 32 * c + p.out_plane] = __float2bfloat16_rn(acc[c] - __bfloat162float(hi));
+  for (int c = 0; c < DPL; ++c) red_o[warp][lane * DPL + c] = acc[c];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int col = threadIdx.x;
+    const float Lt = (red_l[0] + red_l[1]) + (red_l[2] + red_l[3]);
+    const float v = ((red_o[0][col] + red_o[1][col]) + (red_o[2][col] + red_o[3][col])) / Lt;
+    __nv_bfloat16* dst = out + (size_t)m_row * p.n_q * D + j * D + col;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    dst[0] = hi;
+    dst[p.out_plane] = __float2bfloat16_rn(v - __bfloat162float(hi));
   }
 }
 
 cudaError_t launch_attn_gmerge(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {
-  const int warps = p.bs * p.B * p.n_q;
+  const int rows = p.bs * p.B * p.n_q;
   if (p.d == 128)
-    return launch_kernel(attn_gmerge_kernel<128>, dim3((warps + 7) / 8), dim3(256), 0, st, pdl, p,
-                         (__nv_bfloat16*)out);
+    return launch_kernel(attn_gmerge_kernel<128>, dim3(rows), dim3(128), 0, st, pdl, p, (__nv_bfloat16*)out);
   if (p.d == 64)
-    return launch_kernel(attn_gmerge_kernel<64>, dim3((warps + 7) / 8), dim3(256), 0, st, pdl, p,
-                         (__nv_bfloat16*)out);
+    return launch_kernel(attn_gmerge_kernel<64>, dim3(rows), dim3(128), 0, st, pdl, p, (__nv_bfloat16*)out);
   return cudaErrorInvalidValue;
 }
 
@@ -655,8 +662,7 @@ static cudaError_t launch_cluster_t(const AttnParams& p, void* out, cudaStream_t
   cfg.numAttrs = p.n_splits > 1 && !gmerge ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, attn_cluster_kernel<D, NST, KS>, p, (__nv_bfloat16*)out);
   if (e != cudaSuccess || !gmerge) return e;
-  const int warps = p.bs * p.B * p.n_q;
-  return launch_kernel(attn_gmerge_kernel<D>, dim3((warps + 7) / 8), dim3(256), 0, st, pdl, p, (__nv_bfloat16*)out);
+  return launch_attn_gmerge(p, out, st, pdl);
 }
 
 cudaError_t launch_attn_cluster(const AttnParams& p, void* out, cudaStream_t st, bool pdl) {

@@ -287,8 +287,9 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
       // Issue order: the P·V of the oldest softmaxed tile as soon as its P is
       // complete (it frees the tile's ring slot and, once done, its S/P buffer),
       // otherwise the next tile's S once its K/V have landed and the P·V that read
-      // its S/P buffer last is complete. Every try is non-blocking; the time
-      // without progress is bounded.
+      // its S/P buffer last is complete. Every probe is non-blocking (test_wait:
+      // a suspending try_wait on one barrier would hold up work the other allows);
+      // the time without progress is bounded.
       int ns = 0, npv = 0;
       uint64_t idle_since = globaltimer_ns();
       while (ok && npv < n_tiles) {
@@ -296,14 +297,14 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
           ok = false;
           break;
         }
-        if (npv < ns && mbar_try_wait(&p_full[npv % NSB], (npv / NSB) & 1)) {
+        if (npv < ns && mbar_test_wait(&p_full[npv % NSB], (npv / NSB) & 1)) {
           pv(npv++);
           idle_since = globaltimer_ns();
           continue;
         }
         // the S buffer of tile ns held the P of tile ns - NSB: its P·V must be complete
-        if (ns < n_tiles && mbar_try_wait(&kv_full[ns % NST], (ns / NST) & 1) &&
-            (ns < NSB || mbar_try_wait(&pv_done[ns % NSB], ((ns - NSB) / NSB) & 1))) {
+        if (ns < n_tiles && mbar_test_wait(&kv_full[ns % NST], (ns / NST) & 1) &&
+            (ns < NSB || mbar_test_wait(&pv_done[ns % NSB], ((ns - NSB) / NSB) & 1))) {
           tc_fence_after();
           const uint32_t kd = smem_addr(ring + (size_t)(ns % NST) * STAGE);
           const uint32_t qa = smem_addr(qs);
