@@ -98,6 +98,7 @@ struct dflash_ctx {
   size_t att_rows = 0;   // capacity in (split, row) pairs
   int* status = nullptr;
   double* inv_freq = nullptr;   // [head_dim/2] RoPE inverse frequencies
+  float2* rope_cs = nullptr;    // [rows][head_dim/2] (cos, sin) of the current call's row positions
   float* sumsq[2] = {nullptr, nullptr};   // deferred-norm partial sums of squares [H/128][rows], ping-pong
   EncodeTiledFn encode = nullptr;
   bool prof = false;
@@ -377,6 +378,7 @@ GemmSpec spec_qkv(dflash_ctx* ctx, int l, int R, int B, const int* d_ctx_len) {
   qkv.epi.rope_mask = 3u;
   qkv.epi.head_dim = c.head_dim;
   qkv.epi.inv_freq = ctx->inv_freq;
+  qkv.epi.rope_cs = ctx->rope_cs;   // filled for these rows by the call's embedding kernel
   qkv.epi.rows_per_req = B;
   qkv.epi.pos_base = d_ctx_len;
   if (l > 0) set_deferred_norm(ctx, qkv.epi, ctx->sumsq[1], R);   // rows carry the previous layer's norm
@@ -635,6 +637,7 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     const size_t o_attl = take(ctx->att_rows * 4);
     const size_t o_st = take(256);
     const size_t o_freq = take((size_t)c.head_dim / 2 * sizeof(double));
+    const size_t o_rope = take(std::max(R, Rin) * (size_t)(c.head_dim / 2) * sizeof(float2));
     const size_t o_ss0 = take((size_t)(c.hidden / 128) * R * 4);
     const size_t o_ss1 = take((size_t)(c.hidden / 128) * R * 4);
     ctx->ws_bytes = off;
@@ -663,6 +666,7 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     ctx->att_l = (float*)(b + o_attl);
     ctx->status = (int*)(b + o_st);
     ctx->inv_freq = (double*)(b + o_freq);
+    ctx->rope_cs = (float2*)(b + o_rope);
     ctx->sumsq[0] = (float*)(b + o_ss0);
     ctx->sumsq[1] = (float*)(b + o_ss1);
     {
@@ -774,6 +778,8 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
     fcg.epi.out_type = OUT_BF16X2;   // c feeds the K/V GEMM as hi/lo planes
     fcg.epi.out_plane = (size_t)M * c.hidden;
     fcg.epi.rows_per_req = max_new;
+    // side job of the fusion GEMM: the RoPE table of the injected rows' positions
+    fcg.epi.fill = RopeFill{d_start_pos, max_new, M, c.head_dim / 2, ctx->inv_freq, ctx->rope_cs};
     DFL_CHECK(run_gemm(ctx, fcg, st));
 
     // all layers' K and V projections of c, up to kMaxSeg segments per launch
@@ -800,6 +806,7 @@ extern "C" dflash_status dflash_inject_ctx(dflash_ctx* ctx, const void* feats, i
       }
       e.head_dim = c.head_dim;
       e.inv_freq = ctx->inv_freq;
+      e.rope_cs = ctx->rope_cs;
       e.rows_per_req = max_new;
       e.pos_base = d_start_pos;
       e.row_count = d_n_new;
@@ -849,10 +856,12 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
     const double es = (double)esize(ctx);
     {
       ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
+      // the embedding kernel also fills the RoPE table of the block rows' positions
+      const RopeFill rf{d_ctx_len, B, R, c.head_dim / 2, ctx->inv_freq, ctx->rope_cs};
       DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, nullptr, nullptr, B, R,
                                               c.vocab, H,
                                               c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps,
-                                              ctx->x, ctx->h, hb, hb ? (size_t)R * H : 0, ctx->status, st,
+                                              ctx->x, ctx->h, hb, hb ? (size_t)R * H : 0, ctx->status, rf, st,
                                               ctx->use_pdl),
                             "embed_norm launch"));
     }
@@ -1176,9 +1185,10 @@ extern "C" dflash_status dflash_target_forward(dflash_ctx* ctx, const int* d_tok
     const int R = bs * n;
     const int H = c.hidden, KVD = kv_dim(c);
 
+    const RopeFill rf{d_pos0, n, R, c.head_dim / 2, ctx->inv_freq, ctx->rope_cs};
     DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, 0, d_anchor, c.mask_token_id, d_tokens, d_draft, n, R,
                                             c.vocab, H, c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm,
-                                            c.rms_eps, ctx->x, ctx->h, 0, 0, ctx->status, st, ctx->use_pdl),
+                                            c.rms_eps, ctx->x, ctx->h, 0, 0, ctx->status, rf, st, ctx->use_pdl),
                           "embed_norm launch"));
     // The split plan depends on bs and max_ctx only (not on n or the rows' positions),
     // so a row's attention is the same arithmetic in a block forward and in a

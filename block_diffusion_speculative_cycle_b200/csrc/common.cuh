@@ -89,12 +89,40 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // theta^(-2i/d)) at integer position pos. The angle pos*inv_freq is formed and
 // reduced to [-pi, pi] in double (one multiply, one rounding, one fma), so that
 // positions up to 2^24 keep full fp32 accuracy; cos/sin are then taken in fp32.
+// The double arithmetic is slow on this part: the GEMM epilogues read (cos, sin)
+// from a per-row table filled once per call (RopeFill below) instead.
 __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
   const double two_pi = 6.283185307179586;
   const double a = (double)pos * inv_freq;
   const double k = rint(a * (1.0 / two_pi));
   const float r = (float)fma(-k, two_pi, a);
   sincosf(r, s, c);
+}
+
+// The per-row RoPE table of one call: out[m * half + i] = (cos, sin) of the angle
+// of row m's position, pos_base[m / rows_per_req] + m % rows_per_req, at
+// inv_freq[i], for rows m < rows (out null: nothing to fill).
+struct RopeFill {
+  const int* pos_base;
+  int rows_per_req;
+  int rows;
+  int half;
+  const double* inv_freq;
+  float2* out;
+};
+
+__device__ __forceinline__ void rope_fill_entry(const RopeFill& f, int e) {
+  const int m = e / f.half, i = e % f.half;
+  const int pos = __ldg(f.pos_base + m / f.rows_per_req) + m % f.rows_per_req;
+  float c, s;
+  rope_cos_sin(pos, __ldg(f.inv_freq + i), &c, &s);
+  f.out[e] = make_float2(c, s);
+}
+// entries first, first + stride, ... of the whole table
+__device__ __forceinline__ void rope_fill_range(const RopeFill& f, int first, int stride) {
+  if (!f.out) return;
+  const int n = f.rows * f.half;
+  for (int e = first; e < n; e += stride) rope_fill_entry(f, e);
 }
 
 // silu(g) = g * sigmoid(g), with the fast exponential and divide intrinsics

@@ -35,6 +35,8 @@ struct EpiParams {
   unsigned int rope_mask;            // bit s: rotate segment s
   int head_dim;
   const double* inv_freq;            // [head_dim/2] theta^(-2i/d), double
+  const float2* rope_cs;             // [rows][head_dim/2] (cos, sin) of each activation row's position
+  RopeFill fill;                     // side job of this launch: fill the next launch's RoPE table
   int rows_per_req;                  // activation row m belongs to request m / rows_per_req
   const int* pos_base;               // [bs] absolute position of each request's first row
   const int* row_count;              // [bs] valid rows per request (nullptr: all)
@@ -98,8 +100,9 @@ __device__ __forceinline__ void store_out(void* base, size_t idx, float v, int t
   }
 }
 
-// Scratch of the epilogue (shared memory, per CTA): row scales, then a 4 x 32 reduction area.
-constexpr int kEpiScratch = kChunkRows + 4 * kChunkRows;
+// Scratch of the epilogue (shared memory, per CTA): row scales, then an 8 x 32-float
+// reduction area (4 x 32 floats, or 4 x 32 64-bit argmax keys).
+constexpr int kEpiScratch = kChunkRows + 8 * kChunkRows;
 
 // Row scales of the deferred RMSNorm for rows row0 .. row0+nrows-1 into
 // scale[0..nrows): warp w takes rows w, w+4, ...; lane i sums partials i,
@@ -132,15 +135,30 @@ __device__ __forceinline__ void epilogue_row_scales(const EpiParams& e, int row0
 // Apply the epilogue of kind KIND to one staged chunk: acc[j * kChunkLd + t]
 // holds the accumulator of activation row row0 + j (j < nrows) and tile row t
 // (0..127), scaled by rs[j] when the input rows carry a deferred norm (rs is
-// ignored otherwise). red is a [4][kChunkRows] scratch area. Called by 128
-// threads with t = their tile row. The residual epilogue synchronises the 128
-// threads once (named barrier 2) when it produces partial sums of squares. Loops over rows are kept rolled (or lightly unrolled): the
-// epilogue runs once per CTA, so its code is fetched cold and its size, not its
-// instruction count, sets its time.
+// ignored otherwise); the residual epilogue overwrites it. red is a
+// [8][kChunkRows]-float scratch area (8-byte aligned). Called by 128 threads with
+// t = their tile row; the residual and argmax epilogues synchronise the 128
+// threads (named barrier 2).
+// Each of the four epilogue warps runs alone on its scheduler. A chunk of a few
+// rows (the rows one split owns in a split-K cluster) takes a small rolled loop:
+// the code is fetched cold once per CTA and its size sets the time. Wider chunks
+// take kEpiU rows at a time with their loads and long-latency arithmetic issued
+// before any result is used, so no row waits out a full memory or math latency
+// on its own.
+constexpr int kEpiNarrow = 8;
+constexpr int kEpiU = 8;
+
 template <int KIND>
-__device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t,
+__device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, int nrows, float* acc, int t,
                                         const float* rs, float* red) {
   if (!e.norm_part) rs = nullptr;
+  // The launch parameters live in constant memory and are reached through a
+  // reference: copy what the row loops use into registers once, so no global
+  // store inside a loop can force them to be read again.
+  const int out_type = e.out_type;
+  const size_t out_plane = e.out_plane;
+  const int rpr = e.rows_per_req;
+  const int* const pos_base = e.pos_base;
   auto A = [&](int j, int c) -> float {
     const float v = acc[j * kChunkLd + c];
     return rs ? v * rs[j] : v;
@@ -152,20 +170,43 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
     const int d = e.head_dim, half = d >> 1;
     const int jd = n % d;
     const int tp = jd < half ? t + half : t - half;
-    const double f = rope ? __ldg(e.inv_freq + jd % half) : 0.0;
+    // (cos, sin) of row m at this thread's frequency: the call's RoPE table
+    const float2* const cs_col = e.rope_cs + jd % half;
+    void* const out = e.out[s];
+    const size_t ld = (size_t)e.ld_out[s];
+    if (nrows <= kEpiNarrow) {
 #pragma unroll 1
-    for (int j = 0; j < nrows; ++j) {
-      const int m = row0 + j;
-      float v = A(j, t);
-      if (rope) {
-        const int req = m / e.rows_per_req, i = m % e.rows_per_req;
-        const int pos = __ldg(e.pos_base + req) + i;
-        float c, sn;
-        rope_cos_sin(pos, f, &c, &sn);
-        const float w = A(j, tp);
-        v = jd < half ? v * c - w * sn : v * c + w * sn;
+      for (int j = 0; j < nrows; ++j) {
+        const int m = row0 + j;
+        float v = A(j, t);
+        if (rope) {
+          const float2 r = __ldg(cs_col + (size_t)m * half);
+          const float w = A(j, tp);
+          v = jd < half ? v * r.x - w * r.y : v * r.x + w * r.y;
+        }
+        store_out(out, (size_t)m * ld + n, v, out_type, out_plane);
       }
-      store_out(e.out[s], (size_t)m * e.ld_out[s] + n, v, e.out_type, e.out_plane);
+      return;
+    }
+#pragma unroll 1
+    for (int j0 = 0; j0 < nrows; j0 += kEpiU) {
+      float2 r[kEpiU];
+      if (rope) {
+#pragma unroll
+        for (int u = 0; u < kEpiU; ++u) r[u] = __ldg(cs_col + (size_t)(row0 + min(j0 + u, nrows - 1)) * half);
+      }
+#pragma unroll
+      for (int u = 0; u < kEpiU; ++u) {
+        const int j = j0 + u;
+        if (j < nrows) {
+          float v = A(j, t);
+          if (rope) {
+            const float w = A(j, tp);
+            v = jd < half ? v * r[u].x - w * r[u].y : v * r[u].x + w * r[u].y;
+          }
+          store_out(out, (size_t)(row0 + j) * ld + n, v, out_type, out_plane);
+        }
+      }
     }
   } else if constexpr (KIND == EPI_KV_INJECT) {
     const int s = seg_of_tile(e, tile);
@@ -174,63 +215,139 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
     const int d = e.head_dim, half = d >> 1;
     const int jd = n % d, head = n / d;
     const int tp = jd < half ? t + half : t - half;
-    const double f = rope ? __ldg(e.inv_freq + jd % half) : 0.0;
-#pragma unroll 1
-    for (int j = 0; j < nrows; ++j) {
+    const float2* const cs_col = e.rope_cs + jd % half;   // the call's RoPE table, this frequency
+    void* const out = e.out[s];
+    const int cache_type = e.cache_type;
+    const int* const row_count = e.row_count;
+    const int* const page_table = e.page_table;
+    const int max_pages = e.max_pages, num_pages = e.num_pages, page_size = e.page_size, n_kv = e.n_kv;
+    int* const status = e.status;
+    // destination of row j (-1: not stored; a bad position or page is flagged)
+    auto dest = [&](int j, int* pos_out) -> long long {
       const int m = row0 + j;
-      const int req = m / e.rows_per_req, i = m % e.rows_per_req;
-      if (e.row_count && i >= __ldg(e.row_count + req)) continue;
-      const int pos = __ldg(e.pos_base + req) + i;
-      const int slot = pos / e.page_size;
-      if (pos < 0 || slot >= e.max_pages) {
-        if (t == 0) flag_error(e.status, ST_BAD_PAGE);
-        continue;
+      const int req = m / rpr, i = m % rpr;
+      if (j >= nrows || (row_count && i >= __ldg(row_count + req))) return -1;
+      const int ps = __ldg(pos_base + req) + i;
+      const int slot = ps / page_size;
+      if (ps < 0 || slot >= max_pages) {
+        if (t == 0) flag_error(status, ST_BAD_PAGE);
+        return -1;
       }
-      const int page = __ldg(e.page_table + (size_t)req * e.max_pages + slot);
-      if (page < 0 || page >= e.num_pages) {
-        if (t == 0) flag_error(e.status, ST_BAD_PAGE);
-        continue;
+      const int page = __ldg(page_table + (size_t)req * max_pages + slot);
+      if (page < 0 || page >= num_pages) {
+        if (t == 0) flag_error(status, ST_BAD_PAGE);
+        return -1;
       }
-      float v = A(j, t);
+      *pos_out = ps;
+      return (long long)((((size_t)page * n_kv + head) * page_size + (ps % page_size)) * d + jd);
+    };
+    if (nrows <= kEpiNarrow) {
+#pragma unroll 1
+      for (int j = 0; j < nrows; ++j) {
+        int ps = 0;
+        const long long dst = dest(j, &ps);
+        if (dst < 0) continue;
+        float v = A(j, t);
+        if (rope) {
+          const float2 r = __ldg(cs_col + (size_t)(row0 + j) * half);
+          const float w = A(j, tp);
+          v = jd < half ? v * r.x - w * r.y : v * r.x + w * r.y;
+        }
+        store_out(out, (size_t)dst, v, cache_type);
+      }
+      return;
+    }
+#pragma unroll 1
+    for (int j0 = 0; j0 < nrows; j0 += kEpiU) {
+      // destination of each row (-1: not stored), then the rotation
+      long long dst[kEpiU];
+      int pos[kEpiU];
+#pragma unroll
+      for (int u = 0; u < kEpiU; ++u) {
+        pos[u] = 0;
+        dst[u] = dest(j0 + u, &pos[u]);
+      }
+      float2 r[kEpiU];
       if (rope) {
-        float c, sn;
-        rope_cos_sin(pos, f, &c, &sn);
-        const float w = A(j, tp);
-        v = jd < half ? v * c - w * sn : v * c + w * sn;
+#pragma unroll
+        for (int u = 0; u < kEpiU; ++u) r[u] = __ldg(cs_col + (size_t)(row0 + min(j0 + u, nrows - 1)) * half);
       }
-      const size_t dst = (((size_t)page * e.n_kv + head) * e.page_size + (pos % e.page_size)) * d + jd;
-      store_out(e.out[s], dst, v, e.cache_type);
+#pragma unroll
+      for (int u = 0; u < kEpiU; ++u) {
+        if (dst[u] < 0) continue;
+        const int j = j0 + u;
+        float v = A(j, t);
+        if (rope) {
+          const float w = A(j, tp);
+          v = jd < half ? v * r[u].x - w * r[u].y : v * r[u].x + w * r[u].y;
+        }
+        store_out(out, (size_t)dst[u], v, cache_type);
+      }
     }
   } else if constexpr (KIND == EPI_RESID) {
     const int n = tile * kTileN + t;
     const int w = t >> 5, lane = t & 31;
-    const float gn = e.xg ? __ldg(e.gamma_next + n) : 0.f;
-#pragma unroll 4
-    for (int j = 0; j < nrows; ++j) {
-      float* xp = e.x + (size_t)(row0 + j) * e.ldx + n;
-      const float xv = *xp + A(j, t);
-      *xp = xv;
-      if (e.xg) store_out(e.xg, (size_t)(row0 + j) * e.ldx + n, xv * gn, e.out_type, e.out_plane);
-      if (e.sumsq) {
-        const float ss = warp_sum(xv * xv);
-        if (lane == 0) red[w * kChunkRows + j] = ss;
+    float* const x = e.x;
+    const size_t ldx = (size_t)e.ldx;
+    void* const xg = e.xg;
+    float* const sumsq = e.sumsq;
+    const float gn = xg ? __ldg(e.gamma_next + n) : 0.f;
+    if (nrows <= kEpiNarrow) {
+#pragma unroll 1
+      for (int j = 0; j < nrows; ++j) {
+        float* xp = x + (size_t)(row0 + j) * ldx + n;
+        const float xv = *xp + A(j, t);
+        *xp = xv;
+        if (xg) store_out(xg, (size_t)(row0 + j) * ldx + n, xv * gn, out_type, out_plane);
+        if (sumsq) {
+          const float ss = warp_sum(xv * xv);
+          if (lane == 0) red[w * kChunkRows + j] = ss;
+        }
+      }
+    } else {
+      // every row's residual first (independent loads), then add and store; the
+      // squares go back into this thread's own staging slots for the row sums
+      float xo[kChunkRows];
+#pragma unroll
+      for (int j = 0; j < kChunkRows; ++j) xo[j] = j < nrows ? x[(size_t)(row0 + j) * ldx + n] : 0.f;
+#pragma unroll
+      for (int j = 0; j < kChunkRows; ++j) {
+        if (j < nrows) {
+          const float xv = xo[j] + A(j, t);
+          x[(size_t)(row0 + j) * ldx + n] = xv;
+          if (xg) store_out(xg, (size_t)(row0 + j) * ldx + n, xv * gn, out_type, out_plane);
+          acc[j * kChunkLd + t] = xv * xv;
+        }
+      }
+      if (sumsq) {
+        // warp w sums columns 32w .. 32w+31 of row `lane` in column order
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        if (lane < nrows) {
+          const float* r = acc + lane * kChunkLd + 32 * w;
+          float ss = 0.f;
+#pragma unroll 8
+          for (int c = 0; c < 32; ++c) ss += r[c];
+          red[w * kChunkRows + lane] = ss;
+        }
       }
     }
-    if (e.sumsq) {
+    if (sumsq) {
       // this tile's 128 columns of each row: the 4 warp sums in warp order
       asm volatile("bar.sync 2, 128;" ::: "memory");
       if (t < nrows)
-        e.sumsq[(size_t)tile * e.ld_part + row0 + t] =
+        sumsq[(size_t)tile * e.ld_part + row0 + t] =
             red[t] + red[kChunkRows + t] + red[2 * kChunkRows + t] + red[3 * kChunkRows + t];
     }
   } else if constexpr (KIND == EPI_SWIGLU) {
     // column c of the 64 gate / up pairs; the two thread halves take alternate rows
     const int c = t & (kTileN / 2 - 1);
     const int f = tile * (kTileN / 2) + c;
-#pragma unroll 2
+    void* const out = e.out[0];
+    const size_t ld = (size_t)e.ld_out[0];
+#pragma unroll kEpiU
     for (int j = t >> 6; j < nrows; j += 2) {
       const float g = A(j, c), u = A(j, c + kTileN / 2);
-      store_out(e.out[0], (size_t)(row0 + j) * e.ld_out[0] + f, silu_f(g) * u, e.out_type, e.out_plane);
+      store_out(out, (size_t)(row0 + j) * ld + f, silu_f(g) * u, out_type, out_plane);
     }
   } else if constexpr (KIND == EPI_SAMPLE) {
     // warp w takes rows w, w+4, ...; lane scans vocab rows vbase + lane + 32k, k < 4,
@@ -261,27 +378,37 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
       if (lane == 0) atomicMax(e.keys + m, best);
     }
   } else if constexpr (KIND == EPI_ARGMAX) {
-    // warp w takes rows w, w+4, ...; each lane scans 4 of the tile's 128 vocab rows
+    // lane = row of the chunk, warp w = vocab rows 32w .. 32w+31 of the tile (no
+    // shuffles: each thread scans its 32 scores), then the 4 warps' keys of a row
+    // meet in shared memory and one thread per row folds them into keys[m]
     const int w = t >> 5, lane = t & 31;
-    const int vbase = tile * kTileN;
-#pragma unroll 1
-    for (int j = w; j < nrows; j += 4) {
+    const int vbase = tile * kTileN + 32 * w;
+    unsigned long long* red64 = reinterpret_cast<unsigned long long*>(red);
+    if (lane < nrows) {
+      const float* row = acc + lane * kChunkLd + 32 * w;
+      const float sc = rs ? rs[lane] : 1.f;
       unsigned long long best = 0ull;
-#pragma unroll
-      for (int k = 0; k < kTileN / 32; ++k) {
-        const int c = lane + 32 * k;
-        const unsigned long long key = argmax_key(A(j, c), vbase + c);
+#pragma unroll 8
+      for (int c = 0; c < 32; ++c) {
+        const float v = rs ? row[c] * sc : row[c];
+        const unsigned long long key = argmax_key(v, vbase + c);
         best = key > best ? key : best;
       }
-      best = warp_max_u64(best);
-      if (lane == 0) atomicMax(e.keys + row0 + j, best);
+      red64[w * kChunkRows + lane] = best;
+    }
+    asm volatile("bar.sync 2, 128;" ::: "memory");
+    if (t < nrows) {
+      unsigned long long best = red64[t];
+#pragma unroll
+      for (int q = 1; q < 4; ++q) best = red64[q * kChunkRows + t] > best ? red64[q * kChunkRows + t] : best;
+      atomicMax(e.keys + row0 + t, best);
     }
   }
 }
 
 // Runtime dispatch (CUDA-core GEMM): scratch[0..kChunkRows) holds the row scales,
 // the rest the reduction area.
-__device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, int nrows, const float* acc, int t,
+__device__ inline void epilogue_chunk(const EpiParams& e, int tile, int row0, int nrows, float* acc, int t,
                                       float* scratch) {
   const float* rs = scratch;
   float* red = scratch + kChunkRows;

@@ -14,7 +14,7 @@ __global__ void __launch_bounds__(128) gemm_simt_kernel(const GemmSimtParams p) 
   __shared__ float xs[kChunkRows][kKT + 1];
   __shared__ float ws[kTileN][kKT + 1];
   __shared__ float chunk[kChunkRows * kChunkLd];
-  __shared__ float epi_scratch[kEpiScratch];
+  __shared__ __align__(16) float epi_scratch[kEpiScratch];
   const int tile = blockIdx.x;
   const int row0 = blockIdx.y * kChunkRows;
   const int t = threadIdx.x;
@@ -23,6 +23,9 @@ __global__ void __launch_bounds__(128) gemm_simt_kernel(const GemmSimtParams p) 
   const XT* x = reinterpret_cast<const XT*>(p.x);
   grid_dep_wait();
   grid_dep_launch();
+  // side job: this CTA's share of the next launch's RoPE table
+  rope_fill_range(p.epi.fill, ((int)blockIdx.y * (int)gridDim.x + (int)blockIdx.x) * 128 + t,
+                  (int)(gridDim.x * gridDim.y) * 128);
 
   // weight row pointer for tile row r
   auto wrow = [&](int r) -> const WT* {

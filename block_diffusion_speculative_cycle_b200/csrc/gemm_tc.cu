@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
   __shared__ uint64_t stall_bar;   // failure-injection hook only: never arrived at
   __shared__ uint32_t tmem_slot;
   __shared__ int s_flag;
-  __shared__ float epi_scratch[kEpiScratch];
+  __shared__ __align__(16) float epi_scratch[kEpiScratch];
   __shared__ float row_scale[256];   // deferred-norm scales of the tile's activation rows
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -187,6 +187,8 @@ __global__ void __launch_bounds__(kThreads, 3) gemm_tc_kernel(const __grid_const
     grid_dep_wait();   // epilogue reads / writes data shared with the previous kernel
     // the row scales depend only on earlier kernels: compute them while the MMAs run
     epilogue_row_scales(p.epi, row0, rows_here, row_scale, t);
+    // side job, also in the MMAs' shadow: this CTA's share of the next launch's RoPE table
+    rope_fill_range(p.epi.fill, (int)blockIdx.x * 128 + t, (int)gridDim.x * 128);
     bool got = nkb > 0 ? mbar_wait(&acc_bar, 0, status) : true;
     // failure-injection hook: a wait that can only run out (nothing is in flight now)
     if (p.test_stall_ns && got) got = mbar_wait(&stall_bar, 0, status, p.test_stall_ns);

@@ -76,9 +76,10 @@ cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int i
 // position i = m % B): tokens[m] when tokens is given; else the anchor at i = 0 and
 // draft[request, i-1] (when draft is given) or the mask id at i >= 1.
 // With h_plane != 0 (bf16 h), h is written as hi/lo planes h_plane elements apart.
+// Each row's block also fills that row's entries of the RoPE table rf (if rf.out).
 cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, const int* tokens,
                               const int* draft, int B, int R, int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
-                              int* status, cudaStream_t st, bool pdl);
+                              int* status, const RopeFill& rf, cudaStream_t st, bool pdl);
 // h[m] = RMSNorm(x[m]) * gain into h (model dtype) and/or y (fp32); either may be null.
 cudaError_t launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
                            cudaStream_t st, bool pdl);

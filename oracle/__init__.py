@@ -12,6 +12,7 @@ Modules
              speculative loop (for the lossless check)
   sampling -- sampled (temperature > 0) verification and Gumbel-max drafting
   philox  -- the Philox4x32-10 counter-based generator of the draft noise
+  policy  -- acceptance counts and the dynamic block-size choice
 
 Parity status per function (what pins each one, see tests/test_oracle_*.py):
   rms_norm, silu, apply_rope, block_attention, drafter_layer, inject,
@@ -25,4 +26,7 @@ Parity status per function (what pins each one, see tests/test_oracle_*.py):
                               greedy limit, Markov-chain loop, softmax frequencies)
   philox4x32_10, draft_uniforms
                               pinned (published known-answer vectors, layout, moments)
+  acceptance_counts, BlockPolicy
+                              pinned (hand-worked counts, geometric closed form,
+                              brute-force enumeration, simulated convergence, limits)
 """
