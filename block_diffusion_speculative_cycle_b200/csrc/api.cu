@@ -24,6 +24,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 constexpr int kAttnTargetCtas = 296;                   // 2 CTAs per SM on 148 SMs
 constexpr int kAttnTilesPerCta = 8;                    // longest key-tile chain per attention CTA
+constexpr int kAttnAdaptivePairs = 128;                // (request, KV head) pairs from which the device picks the split size
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -68,6 +69,8 @@ struct dflash_ctx {
   int attn_form = -1;           // DFLASH_ATTN_FORM=full|compact: force the tcgen05 attention form (experiments)
   int attn_l2promo = 3;         // DFLASH_ATTN_L2PROMO=0..3: L2 promotion of the attention's tensor maps (experiments)
   int attn_stages = 5;          // K/V ring depth of the tcgen05 attention (DFLASH_ATTN_STAGES, experiments)
+  int attn_plan = -1;           // DFLASH_ATTN_PLAN=host|device: force the host's or the device-side split plan
+  int* attn_kps = nullptr;      // the device-side split size of the current draft call
   // GEMM sites (bit 1 kv, 2 qkv, 3 o, 4 gate/up, 5 down) that read their activations
   // as one bf16 plane from single_plane_rows rows on (DFLASH_SINGLE_PLANE=mask,rows)
   unsigned single_plane_mask = 0;
@@ -565,6 +568,8 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
         ctx->single_plane_rows = rows;
       }
     }
+    env = std::getenv("DFLASH_ATTN_PLAN");
+    if (env) ctx->attn_plan = std::strcmp(env, "device") == 0 ? 1 : (std::strcmp(env, "host") == 0 ? 0 : -1);
     env = std::getenv("DFLASH_ATTN_STAGES");
     if (env && std::atoi(env) >= 2 && std::atoi(env) <= kMaxAttnTcStages) ctx->attn_stages = std::atoi(env);
     if (c.head_dim == 128 && ctx->attn_stages > 5) ctx->attn_stages = 5;   // what fits beside Q and P
@@ -616,6 +621,9 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     const int g = c.n_q_heads / c.n_kv_heads;
     const size_t nr = (size_t)g * c.max_block;
     ctx->att_rows = ((size_t)kAttnTargetCtas + (size_t)c.max_batch * c.n_kv_heads + 8) * nr;
+    // the device-side plan's grid: up to 8 waves of two CTAs per SM
+    if ((size_t)c.max_batch * c.n_kv_heads >= (size_t)kAttnAdaptivePairs)
+      ctx->att_rows = std::max(ctx->att_rows, (size_t)16 * ctx->num_sms * nr);
     size_t off = 0;
     auto take = [&](size_t bytes) {
       size_t o = off;
@@ -636,6 +644,7 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     const size_t o_attm = take(ctx->att_rows * 4);
     const size_t o_attl = take(ctx->att_rows * 4);
     const size_t o_st = take(256);
+    const size_t o_kps = take(256);
     const size_t o_freq = take((size_t)c.head_dim / 2 * sizeof(double));
     const size_t o_rope = take(std::max(R, Rin) * (size_t)(c.head_dim / 2) * sizeof(float2));
     const size_t o_ss0 = take((size_t)(c.hidden / 128) * R * 4);
@@ -665,6 +674,7 @@ extern "C" dflash_status dflash_create(const dflash_config* cfg, const dflash_we
     ctx->att_m = (float*)(b + o_attm);
     ctx->att_l = (float*)(b + o_attl);
     ctx->status = (int*)(b + o_st);
+    ctx->attn_kps = (int*)(b + o_kps);
     ctx->inv_freq = (double*)(b + o_freq);
     ctx->rope_cs = (float2*)(b + o_rope);
     ctx->sumsq[0] = (float*)(b + o_ss0);
@@ -854,17 +864,6 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
     const size_t layer_stride = (size_t)R * H;
 
     const double es = (double)esize(ctx);
-    {
-      ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
-      // the embedding kernel also fills the RoPE table of the block rows' positions
-      const RopeFill rf{d_ctx_len, B, R, c.head_dim / 2, ctx->inv_freq, ctx->rope_cs};
-      DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, nullptr, nullptr, B, R,
-                                              c.vocab, H,
-                                              c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps,
-                                              ctx->x, ctx->h, hb, hb ? (size_t)R * H : 0, ctx->status, rf, st,
-                                              ctx->use_pdl),
-                            "embed_norm launch"));
-    }
     const double norm_bytes = (double)R * H * (4 + es);
 
     // attention split plan. The context of the longest request is cut into n_splits
@@ -917,6 +916,7 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
     const bool attn_tc = ctx->bf16 && ctx->cache_f16 && !ctx->attn_mma && c.page_size % 64 == 0 && g * B <= 128 &&
                          (c.head_dim == 64 || c.head_dim == 128);
     bool attn_compact = false;
+    AttnKpsPlan kplan{};   // out == null: the host's split size
     if (attn_tc) {
       const int nr = g * B;
       const int blk_tiles = (B + 63) / 64;
@@ -971,14 +971,53 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
         }
       }
       if (best >= 1e30) return DFLASH_ERR_UNSUPPORTED;
+      // Many (request, KV head) pairs: the batch's contexts are usually ragged, and
+      // a plan for the longest request leaves most CTA slots idle behind it. The
+      // global merge then takes a split size that the device picks from the actual
+      // context lengths (the embedding kernel, AttnKpsPlan): about three CTAs with
+      // keys per CTA slot, all with the same number of key tiles. The grid covers
+      // the smallest split size allowed; CTAs past a request's keys exit at once.
+      const bool adaptive = ctx->attn_plan == 1 || (ctx->attn_plan < 0 && pairs >= kAttnAdaptivePairs);
+      if (adaptive) {
+        const int slots = (want_form == 1 ? 2 : 1) * ctx->num_sms;
+        const int keys = span + B;   // a request's keys: its (window of) context and the block
+        const int key_tiles = (keys + 63) / 64;
+        int min_tiles =
+            std::max(4, (int)(((long long)pairs * key_tiles + 8LL * slots - 1) / (8LL * slots)));   // grid <= 8 waves
+        int sp = (keys + 64 * min_tiles - 1) / (64 * min_tiles);
+        while ((size_t)pairs * sp * nr > ctx->att_rows && sp > 1) {
+          ++min_tiles;
+          sp = (keys + 64 * min_tiles - 1) / (64 * min_tiles);
+        }
+        if ((size_t)pairs * sp * nr <= ctx->att_rows) {
+          kplan = AttnKpsPlan{d_ctx_len, bs, B, c.window, max_ctx, min_tiles,
+                              std::max(1, 3 * slots / c.n_kv_heads), ctx->attn_kps};
+          n_splits = std::max(1, sp);
+          kps = 64 * min_tiles;
+          attn_gmerge = true;
+          attn_compact = want_form == 1;
+        }
+      }
     }
     if (ctx->debug)
-      std::fprintf(stderr, "dflash attention %s%s pairs=%d splits=%d kps=%d gmerge=%d span=%d\n",
+      std::fprintf(stderr, "dflash attention %s%s pairs=%d splits=%d kps=%d gmerge=%d span=%d%s\n",
                    attn_tc ? "tcgen05" : (ctx->bf16 ? "mma.sync" : "simt"), attn_compact ? " compact" : "", pairs,
-                   n_splits, kps, (int)attn_gmerge, span);
+                   n_splits, kps, (int)attn_gmerge, span, kplan.out ? " (split size chosen on the device)" : "");
     // split partials in global memory (CUDA-core path, or the global merge) must fit the workspace
     if ((!ctx->bf16 || attn_gmerge) && (size_t)bs * c.n_kv_heads * n_splits * g * B > ctx->att_rows)
       return DFLASH_ERR_UNSUPPORTED;
+    {
+      ProfScope prof(ctx, PK_EMBED_NORM, st, (double)R * H * (es + 4 + es), 0);
+      // the embedding kernel also fills the RoPE table of the block rows' positions
+      // (and, for the device-side attention plan, the call's split size)
+      const RopeFill rf{d_ctx_len, B, R, c.head_dim / 2, ctx->inv_freq, ctx->rope_cs};
+      DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, hb, d_anchor, c.mask_token_id, nullptr, nullptr, B, R,
+                                              c.vocab, H,
+                                              c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm, c.rms_eps,
+                                              ctx->x, ctx->h, hb, hb ? (size_t)R * H : 0, ctx->status, rf, kplan, st,
+                                              ctx->use_pdl),
+                            "embed_norm launch"));
+    }
 
     for (int l = 0; l < c.n_layers; ++l) {
       DFL_CHECK(run_gemm(ctx, spec_qkv(ctx, l, R, B, d_ctx_len), st));
@@ -1004,6 +1043,7 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
       ap.n_splits = n_splits;
       ap.ks = attn_ks;
       ap.global_merge = attn_gmerge ? 1 : 0;
+      ap.kps_dev = kplan.out;
       ap.max_ctx = max_ctx;
       ap.window = c.window;
       ap.scale = (float)(1.0 / std::sqrt((double)c.head_dim));
@@ -1188,7 +1228,8 @@ extern "C" dflash_status dflash_target_forward(dflash_ctx* ctx, const int* d_tok
     const RopeFill rf{d_pos0, n, R, c.head_dim / 2, ctx->inv_freq, ctx->rope_cs};
     DFL_CHECK(cuda_status(launch_embed_norm(ctx->embed, 0, d_anchor, c.mask_token_id, d_tokens, d_draft, n, R,
                                             c.vocab, H, c.n_layers > 0 ? ctx->attn_norm[0] : ctx->final_norm,
-                                            c.rms_eps, ctx->x, ctx->h, 0, 0, ctx->status, rf, st, ctx->use_pdl),
+                                            c.rms_eps, ctx->x, ctx->h, 0, 0, ctx->status, rf, AttnKpsPlan{}, st,
+                                            ctx->use_pdl),
                           "embed_norm launch"));
     // The split plan depends on bs and max_ctx only (not on n or the rows' positions),
     // so a row's attention is the same arithmetic in a block forward and in a

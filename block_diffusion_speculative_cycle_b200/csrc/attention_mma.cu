@@ -574,7 +574,8 @@ __global__ void __launch_bounds__(128) attn_gmerge_kernel(const AttnParams p, __
   const int nr = p.g * p.B, r = jj * p.B + i;
   int P = p.ctx_len[b];
   P = P < 0 ? 0 : (P > p.max_ctx ? p.max_ctx : P);
-  const int used = min(p.n_splits, (P + p.B - attn_key_base(attn_ctx_lo(P, p.window)) + p.kps - 1) / p.kps);
+  const int kps = attn_kps(p);
+  const int used = min(p.n_splits, (P + p.B - attn_key_base(attn_ctx_lo(P, p.window)) + kps - 1) / kps);
   const size_t base = (size_t)(b * p.n_kv + h) * p.n_splits * nr + r;
   // the row's maximum over the splits
   float M = -INFINITY;

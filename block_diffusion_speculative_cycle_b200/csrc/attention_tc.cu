@@ -132,8 +132,9 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
   const int S = p.n_splits;
   const int T_all = P + p.B;
   const int ctx_lo = attn_ctx_lo(P, p.window);
-  const int k0 = min(T_all, attn_key_base(ctx_lo) + s * p.kps);
-  const int k1 = s == S - 1 ? T_all : min(T_all, k0 + p.kps);
+  const int kps = attn_kps(p);   // the host's, or the call's device-side plan (global merge)
+  const int k0 = min(T_all, attn_key_base(ctx_lo) + s * kps);
+  const int k1 = s == S - 1 ? T_all : min(T_all, k0 + kps);
   const int cx1 = min(k1, P);                               // context part [k0, cx1)
   const int n_ctx = cx1 > k0 ? (cx1 - k0 + kKT - 1) / kKT : 0;
   const int bk0 = max(k0, P) - P, bk1 = k1 - P;             // block rows [bk0, bk1)

@@ -29,7 +29,25 @@ struct AttnParams {
   int global_merge;           // tensor-core path: splits write part_o/m/l (exp2 domain) and a second kernel merges
   int window;                 // sliding window: the block sees context positions P-window .. P-1 only (0: all)
   int causal;                 // fp32 path only: block row i sees block keys 0..i (a causal decoder), not all B
+  // Global merge with a split size chosen on the device (tensor-core path; null:
+  // kps above): the keys per split, written by the call's embedding kernel from
+  // every request's actual context length (AttnKpsPlan).
+  const int* kps_dev;
 };
+
+// The device-side split size of a batch: with T = the key tiles of all requests
+// (each request: its window's 64-aligned start to P, plus the B block keys),
+// kps = 64 * max(min_tiles, ceil(T / target_items)), so that the CTAs that have
+// keys (target_items per KV head) carry equal work however ragged the batch is.
+struct AttnKpsPlan {
+  const int* ctx_len;   // [bs]
+  int bs, B, window, max_ctx;
+  int min_tiles, target_items;
+  int* out;             // null: no plan this call
+};
+
+// Keys per split of the call (kps_dev set), else the host's.
+__device__ __forceinline__ int attn_kps(const AttnParams& p) { return p.kps_dev ? __ldg(p.kps_dev) : p.kps; }
 
 // First context key the block attends to, and the 64-aligned key where split 0
 // starts (keys from there up to ctx_lo are masked; a 64-key tile never crosses a
@@ -76,10 +94,11 @@ cudaError_t launch_attention(const AttnParams& p, void* out, int out_bf16, int i
 // position i = m % B): tokens[m] when tokens is given; else the anchor at i = 0 and
 // draft[request, i-1] (when draft is given) or the mask id at i >= 1.
 // With h_plane != 0 (bf16 h), h is written as hi/lo planes h_plane elements apart.
-// Each row's block also fills that row's entries of the RoPE table rf (if rf.out).
+// Each row's block also fills that row's entries of the RoPE table rf (if rf.out);
+// block 0 also computes the call's attention split size (kp.out, if set).
 cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, const int* tokens,
                               const int* draft, int B, int R, int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
-                              int* status, const RopeFill& rf, cudaStream_t st, bool pdl);
+                              int* status, const RopeFill& rf, const AttnKpsPlan& kp, cudaStream_t st, bool pdl);
 // h[m] = RMSNorm(x[m]) * gain into h (model dtype) and/or y (fp32); either may be null.
 cudaError_t launch_rmsnorm(const float* x, int R, int H, const float* gain, float eps, void* h, int h_bf16, float* y,
                            cudaStream_t st, bool pdl);

@@ -79,11 +79,27 @@ template <int VPT, typename ET, typename HT>
 __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const ET* embed, const int* anchor, int mask_id,
                                                                   const int* tokens, const int* draft, int B, int V,
                                                                   int H, const float* gain, float eps, float* x, HT* h,
-                                                                  size_t h_plane, int* status, const RopeFill rf) {
+                                                                  size_t h_plane, int* status, const RopeFill rf,
+                                                                  const AttnKpsPlan kp) {
   __shared__ float red[32];
   grid_dep_wait();
   grid_dep_launch();
   const int m = blockIdx.x;
+  if (kp.out && m == 0 && threadIdx.x < 32) {
+    // the attention split size of this call, from every request's key tiles
+    int tiles = 0;
+    for (int r = threadIdx.x; r < kp.bs; r += 32) {
+      int P = kp.ctx_len[r];
+      P = P < 0 ? 0 : (P > kp.max_ctx ? kp.max_ctx : P);
+      tiles += (P + kp.B - attn_key_base(attn_ctx_lo(P, kp.window)) + 63) / 64;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
+    if (threadIdx.x == 0) {
+      const int per = (tiles + kp.target_items - 1) / kp.target_items;
+      *kp.out = 64 * (per > kp.min_tiles ? per : kp.min_tiles);
+    }
+  }
   // this row's entries of the call's RoPE table (read by the QKV epilogues)
   if (rf.out)
     for (int i = threadIdx.x; i < rf.half; i += blockDim.x) rope_fill_entry(rf, m * rf.half + i);
@@ -141,38 +157,39 @@ __global__ void argmax_finalize_kernel(unsigned long long* keys, int bs, int B, 
 template <int VPT>
 static cudaError_t embed_norm_vpt(const void* embed, int embed_bf16, const int* anchor, int mask_id,
                                   const int* tokens, const int* draft, int B, int R, int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16,
-                                  size_t h_plane, int* status, const RopeFill& rf, cudaStream_t st, bool pdl) {
+                                  size_t h_plane, int* status, const RopeFill& rf, const AttnKpsPlan& kp,
+                                  cudaStream_t st, bool pdl) {
   const dim3 g(R), b(kNormThreads);
   if (embed_bf16 && h_bf16)
     return launch_kernel(embed_norm_kernel<VPT, __nv_bfloat16, __nv_bfloat16>, g, b, 0, st, pdl,
                          (const __nv_bfloat16*)embed, anchor, mask_id, tokens, draft, B, V, H, gain, eps, x, (__nv_bfloat16*)h,
-                         h_plane, status, rf);
+                         h_plane, status, rf, kp);
   if (!embed_bf16 && !h_bf16)
     return launch_kernel(embed_norm_kernel<VPT, float, float>, g, b, 0, st, pdl, (const float*)embed, anchor,
-                         mask_id, tokens, draft, B, V, H, gain, eps, x, (float*)h, (size_t)0, status, rf);
+                         mask_id, tokens, draft, B, V, H, gain, eps, x, (float*)h, (size_t)0, status, rf, kp);
   if (embed_bf16)
     return launch_kernel(embed_norm_kernel<VPT, __nv_bfloat16, float>, g, b, 0, st, pdl,
                          (const __nv_bfloat16*)embed, anchor, mask_id, tokens, draft, B, V, H, gain, eps, x, (float*)h, (size_t)0,
-                         status, rf);
+                         status, rf, kp);
   return launch_kernel(embed_norm_kernel<VPT, float, __nv_bfloat16>, g, b, 0, st, pdl, (const float*)embed, anchor,
-                       mask_id, tokens, draft, B, V, H, gain, eps, x, (__nv_bfloat16*)h, h_plane, status, rf);
+                       mask_id, tokens, draft, B, V, H, gain, eps, x, (__nv_bfloat16*)h, h_plane, status, rf, kp);
 }
 
 cudaError_t launch_embed_norm(const void* embed, int embed_bf16, const int* anchor, int mask_id, const int* tokens,
                               const int* draft, int B, int R, int V, int H, const float* gain, float eps, float* x, void* h, int h_bf16, size_t h_plane,
-                              int* status, const RopeFill& rf, cudaStream_t st, bool pdl) {
+                              int* status, const RopeFill& rf, const AttnKpsPlan& kp, cudaStream_t st, bool pdl) {
   const int vpt = (H / 4 + kNormThreads - 1) / kNormThreads;
   if (vpt <= 1)
     return embed_norm_vpt<1>(embed, embed_bf16, anchor, mask_id, tokens, draft, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
-                             rf, st, pdl);
+                             rf, kp, st, pdl);
   if (vpt <= 2)
     return embed_norm_vpt<2>(embed, embed_bf16, anchor, mask_id, tokens, draft, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
-                             rf, st, pdl);
+                             rf, kp, st, pdl);
   if (vpt <= 4)
     return embed_norm_vpt<4>(embed, embed_bf16, anchor, mask_id, tokens, draft, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
-                             rf, st, pdl);
+                             rf, kp, st, pdl);
   return embed_norm_vpt<8>(embed, embed_bf16, anchor, mask_id, tokens, draft, B, R, V, H, gain, eps, x, h, h_bf16, h_plane, status,
-                           rf, st, pdl);
+                           rf, kp, st, pdl);
 }
 
 template <int VPT>

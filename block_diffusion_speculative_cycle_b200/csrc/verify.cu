@@ -31,6 +31,7 @@ __device__ __forceinline__ unsigned long long chunk_best<__nv_bfloat16>(const __
   if (vec) {
     const int nvec = (v1 - v0) / 8;
     const uint4* p = reinterpret_cast<const uint4*>(row + v0);
+#pragma unroll 4
     for (int e = threadIdx.x; e < nvec; e += blockDim.x) {
       const uint4 u = __ldcs(p + e);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -60,6 +61,7 @@ __device__ __forceinline__ unsigned long long chunk_best<float>(const float* row
   if (vec) {
     const int nvec = (v1 - v0) / 4;
     const float4* p = reinterpret_cast<const float4*>(row + v0);
+#pragma unroll 4
     for (int e = threadIdx.x; e < nvec; e += blockDim.x) {
       const float4 f = __ldcs(p + e);
       const float w[4] = {f.x, f.y, f.z, f.w};
@@ -83,6 +85,7 @@ __global__ void __launch_bounds__(kVerifyThreads) verify_kernel(const T* logits,
                                                                  unsigned long long* keys, int* tickets,
                                                                  int* accepted, int* next_token) {
   __shared__ unsigned long long red[kVerifyThreads / 32];
+  __shared__ int s_last;
   grid_dep_wait();
   grid_dep_launch();
   const int c = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
@@ -97,18 +100,32 @@ __global__ void __launch_bounds__(kVerifyThreads) verify_kernel(const T* logits,
     atomicMax(keys + (size_t)b * B + j, best);
     __threadfence();
     const int total = (int)gridDim.x * B;
-    const int prev = atomicAdd(tickets + b, 1);
-    if (prev == total - 1) {
-      __threadfence();
-      unsigned long long* kb = keys + (size_t)b * B;
-      int a = 0;
-      while (a < B - 1 && draft[(size_t)b * (B - 1) + a] == argmax_key_index(__ldcg(kb + a))) ++a;
-      accepted[b] = a;
-      next_token[b] = argmax_key_index(__ldcg(kb + a));
-      for (int r = 0; r < B; ++r) kb[r] = 0ull;
-      tickets[b] = 0;
-    }
+    s_last = atomicAdd(tickets + b, 1) == total - 1;
   }
+  __syncthreads();
+  if (!s_last || warp != 0) return;
+  // the request's last CTA: warp 0 tests 32 drafts per round trip. Lane i of a
+  // round compares draft i with the argmax of row i; a = the leading matches.
+  __threadfence();
+  unsigned long long* kb = keys + (size_t)b * B;
+  const int* dr = draft + (size_t)b * (B - 1);
+  int a = 0;
+  for (int i0 = 0; i0 < B - 1; i0 += 32) {
+    const int i = i0 + lane, nv = min(32, B - 1 - i0);
+    const bool match = i < B - 1 && __ldg(dr + i) == argmax_key_index(__ldcg(kb + i));
+    const unsigned miss = ~__ballot_sync(0xffffffffu, match);
+    const int lead = miss ? __ffs((int)miss) - 1 : 32;   // lanes >= nv count as misses
+    a += lead;
+    if (lead < nv) break;
+  }
+  if (lane == 0) {
+    accepted[b] = a;
+    next_token[b] = argmax_key_index(__ldcg(kb + a));
+  }
+  __syncwarp();
+  // leave the request's keys and ticket zeroed for the next call
+  for (int r = lane; r < B; r += 32) kb[r] = 0ull;
+  if (lane == 0) tickets[b] = 0;
 }
 
 // Programmatic dependent launch for verify (on unless DFLASH_PDL=0).

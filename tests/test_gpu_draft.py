@@ -105,14 +105,28 @@ def test_small_bf16_fp16_cache_long_contexts():
     run_case(SMALL_BF16, lens, 16, seed=9, cache_dtype=torch.float16)
 
 
-@pytest.mark.parametrize("cfg,cache_dtype", [(synth.TINY, None), (SMALL_BF16, None), (SMALL_BF16, torch.float16)],
-                         ids=["fp32-simt", "bf16-mma", "fp16-tcgen05"])
+@pytest.mark.parametrize("plan", ["host", "device"])
+def test_attention_split_plans_on_a_ragged_batch(plan, monkeypatch):
+    """Both split plans of the tcgen05 attention on one ragged batch (an empty
+    context, one key, a page boundary, a few thousand keys): the host's plan for
+    the longest request (cluster merge), and the split size the device picks from
+    the actual context lengths (global merge; CTAs past a request's keys exit)."""
+    monkeypatch.setenv("DFLASH_ATTN_PLAN", plan)
+    lens = [0, 1, 64, 3000, 777, 2048, 130, 1500]
+    run_case(SMALL_BF16, lens, 16, seed=12, cache_dtype=torch.float16)
+
+
+@pytest.mark.parametrize("cfg,cache_dtype,plan",
+                         [(synth.TINY, None, "host"), (SMALL_BF16, None, "host"), (SMALL_BF16, torch.float16, "host"),
+                          (SMALL_BF16, torch.float16, "device")],
+                         ids=["fp32-simt", "bf16-mma", "fp16-tcgen05", "fp16-tcgen05-device-plan"])
 @pytest.mark.parametrize("window", [128, 100])
-def test_sliding_window_matches_the_oracle_with_released_pages(cfg, cache_dtype, window):
+def test_sliding_window_matches_the_oracle_with_released_pages(cfg, cache_dtype, plan, window, monkeypatch):
     """Sliding-window drafting: each request's block sees its last `window` context
     positions. After injection the page-table slots wholly below every window are
     set to -1 (pages released): the pass must not read them, flag nothing, and
     match the oracle's windowed pass."""
+    monkeypatch.setenv("DFLASH_ATTN_PLAN", plan)
     ctx_lens, B, page = [300, 50, 700, 129], 16, 64
     bs = len(ctx_lens)
     ctx = torch.tensor(ctx_lens, dtype=torch.int32)
