@@ -24,7 +24,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 constexpr int kAttnTargetCtas = 296;                   // 2 CTAs per SM on 148 SMs
 constexpr int kAttnTilesPerCta = 8;                    // longest key-tile chain per attention CTA
-constexpr int kAttnAdaptivePairs = 128;                // (request, KV head) pairs from which the device picks the split size
+constexpr int kAttnAdaptivePairs = 64;                 // (request, KV head) pairs from which the device picks the split size
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -974,9 +974,9 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
       // Many (request, KV head) pairs: the batch's contexts are usually ragged, and
       // a plan for the longest request leaves most CTA slots idle behind it. The
       // global merge then takes a split size that the device picks from the actual
-      // context lengths (the embedding kernel, AttnKpsPlan): about three CTAs with
-      // keys per CTA slot, all with the same number of key tiles. The grid covers
-      // the smallest split size allowed; CTAs past a request's keys exit at once.
+      // context lengths (the embedding kernel, AttnKpsPlan: fewest waves x CTA
+      // time). The flat grid covers the smallest split size allowed, items in
+      // order; CTAs past the batch's items come last and exit at once.
       const bool adaptive = ctx->attn_plan == 1 || (ctx->attn_plan < 0 && pairs >= kAttnAdaptivePairs);
       if (adaptive) {
         const int slots = (want_form == 1 ? 2 : 1) * ctx->num_sms;
@@ -990,8 +990,7 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
           sp = (keys + 64 * min_tiles - 1) / (64 * min_tiles);
         }
         if ((size_t)pairs * sp * nr <= ctx->att_rows) {
-          kplan = AttnKpsPlan{d_ctx_len, bs, B, c.window, max_ctx, min_tiles,
-                              std::max(1, 3 * slots / c.n_kv_heads), ctx->attn_kps};
+          kplan = AttnKpsPlan{d_ctx_len, bs, B, c.window, max_ctx, min_tiles, slots, c.n_kv_heads, ctx->attn_kps};
           n_splits = std::max(1, sp);
           kps = 64 * min_tiles;
           attn_gmerge = true;

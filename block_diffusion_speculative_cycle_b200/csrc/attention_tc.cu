@@ -116,10 +116,52 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
   uint8_t* qs = base;
   uint8_t* ring = qs + HALVES * QH;
 
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nr = p.g * p.B;
   int* status = p.status;
+  const int kps = attn_kps(p);   // the host's, or the call's device-side plan (global merge)
+  int s, h, b;
+  if (p.kps_dev) {
+    // Device-side plan: the grid is flat, KV head fastest, then the batch's
+    // (request, split) items in order, so that the CTAs with keys come first and
+    // the ones past the batch's items (launched last) exit at once. Every warp
+    // finds its item's request by a scan of the requests' split counts.
+    h = blockIdx.x % p.n_kv;
+    const int item = blockIdx.x / p.n_kv;
+    if (item >= __ldg(p.kps_dev + 1)) return;   // past the batch's items
+    b = -1;
+    s = 0;
+    for (int r0 = 0, before = 0; r0 < p.bs; r0 += 32) {
+      const int r = r0 + lane;
+      int n = 0;
+      if (r < p.bs) {
+        int Pr = p.ctx_len[r];
+        Pr = Pr < 0 ? 0 : (Pr > p.max_ctx ? p.max_ctx : Pr);
+        n = min(p.n_splits, (Pr + p.B - attn_key_base(attn_ctx_lo(Pr, p.window)) + kps - 1) / kps);
+      }
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int excl = incl - n;
+      const unsigned hit = __ballot_sync(0xffffffffu, r < p.bs && item >= before + excl && item < before + incl);
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (hit) {
+        const int src = __ffs((int)hit) - 1;
+        b = r0 + src;
+        s = item - before - __shfl_sync(0xffffffffu, excl, src);
+        break;
+      }
+      before += total;
+    }
+    if (b < 0) return;   // past the batch's items
+  } else {
+    s = blockIdx.x;
+    h = blockIdx.y;
+    b = blockIdx.z;
+  }
 
   int P = p.ctx_len[b];
   if (P < 0 || P > p.max_ctx) {
@@ -132,7 +174,6 @@ __global__ void __launch_bounds__(tc_threads(COMPACT), COMPACT ? 2 : 1)
   const int S = p.n_splits;
   const int T_all = P + p.B;
   const int ctx_lo = attn_ctx_lo(P, p.window);
-  const int kps = attn_kps(p);   // the host's, or the call's device-side plan (global merge)
   const int k0 = min(T_all, attn_key_base(ctx_lo) + s * kps);
   const int k1 = s == S - 1 ? T_all : min(T_all, k0 + kps);
   const int cx1 = min(k1, P);                               // context part [k0, cx1)
@@ -611,7 +652,8 @@ cudaError_t launch_attn_tc(const AttnTcParams& tp, void* out, cudaStream_t st, b
   cudaError_t e = attn_tc_prepare(p.d, compact, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_splits, p.n_kv, p.bs);
+  // device-side plan: one flat grid over (request, split) items x KV heads
+  cfg.gridDim = p.kps_dev ? dim3((unsigned)(p.n_splits * p.n_kv * p.bs), 1, 1) : dim3(p.n_splits, p.n_kv, p.bs);
   cfg.blockDim = dim3(tc_threads(compact));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;

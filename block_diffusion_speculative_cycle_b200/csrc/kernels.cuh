@@ -30,21 +30,25 @@ struct AttnParams {
   int window;                 // sliding window: the block sees context positions P-window .. P-1 only (0: all)
   int causal;                 // fp32 path only: block row i sees block keys 0..i (a causal decoder), not all B
   // Global merge with a split size chosen on the device (tensor-core path; null:
-  // kps above): the keys per split, written by the call's embedding kernel from
-  // every request's actual context length (AttnKpsPlan).
+  // kps above): [keys per split, the batch's (request, split) items], written by
+  // the call's embedding kernel from every request's context length (AttnKpsPlan).
   const int* kps_dev;
 };
 
-// The device-side split size of a batch: with T = the key tiles of all requests
-// (each request: its window's 64-aligned start to P, plus the B block keys),
-// kps = 64 * max(min_tiles, ceil(T / target_items)), so that the CTAs that have
-// keys (target_items per KV head) carry equal work however ragged the batch is.
+// The device-side split size of a batch, from every request's key tiles t_r (its
+// window's 64-aligned start to P, plus the B block keys): among candidate sizes c
+// (the longest request cut into 1..16 parts, and the batch's tiles spread over
+// 1..4 waves of CTA slots), the one with the fewest waves x (start-up + c tiles),
+// waves = ceil(n_kv * sum_r ceil(t_r / c) / slots); never below min_tiles, which
+// bounds the grid. Ragged batches get short, equal CTAs; uniform ones one wave.
 struct AttnKpsPlan {
   const int* ctx_len;   // [bs]
   int bs, B, window, max_ctx;
-  int min_tiles, target_items;
-  int* out;             // null: no plan this call
+  int min_tiles;        // smallest split (key tiles) the grid and workspace allow
+  int slots, n_kv;      // CTAs resident at once; KV heads (CTAs per item)
+  int* out;             // [2]: keys per split, the batch's (request, split) items; null: no plan
 };
+constexpr int kAttnPlanStartTiles = 4;   // a CTA's start-up (Q, first tiles, merge) in key tiles
 
 // Keys per split of the call (kps_dev set), else the host's.
 __device__ __forceinline__ int attn_kps(const AttnParams& p) { return p.kps_dev ? __ldg(p.kps_dev) : p.kps; }

@@ -86,18 +86,45 @@ __global__ void __launch_bounds__(kNormThreads) embed_norm_kernel(const ET* embe
   grid_dep_launch();
   const int m = blockIdx.x;
   if (kp.out && m == 0 && threadIdx.x < 32) {
-    // the attention split size of this call, from every request's key tiles
-    int tiles = 0;
-    for (int r = threadIdx.x; r < kp.bs; r += 32) {
+    // the attention split size of this call (AttnKpsPlan), one warp
+    const int lane = threadIdx.x;
+    auto tiles_of = [&](int r) {
       int P = kp.ctx_len[r];
       P = P < 0 ? 0 : (P > kp.max_ctx ? kp.max_ctx : P);
-      tiles += (P + kp.B - attn_key_base(attn_ctx_lo(P, kp.window)) + 63) / 64;
+      return (P + kp.B - attn_key_base(attn_ctx_lo(P, kp.window)) + 63) / 64;
+    };
+    int sum_t = 0, max_t = 0;
+    for (int r = lane; r < kp.bs; r += 32) {
+      const int t = tiles_of(r);
+      sum_t += t;
+      max_t = max(max_t, t);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, o);
-    if (threadIdx.x == 0) {
-      const int per = (tiles + kp.target_items - 1) / kp.target_items;
-      *kp.out = 64 * (per > kp.min_tiles ? per : kp.min_tiles);
+    for (int o = 16; o > 0; o >>= 1) {
+      sum_t += __shfl_xor_sync(0xffffffffu, sum_t, o);
+      max_t = max(max_t, __shfl_xor_sync(0xffffffffu, max_t, o));
+    }
+    const int per_head = max(1, kp.slots / kp.n_kv);
+    long long best_cost = -1;
+    int best = max(kp.min_tiles, max_t), best_items = 0;
+    for (int cand = 0; cand < 20; ++cand) {
+      int c = cand < 16 ? (max_t + cand) / (cand + 1) : (sum_t + (cand - 15) * per_head - 1) / ((cand - 15) * per_head);
+      c = max(kp.min_tiles, max(1, c));
+      int items = 0;
+      for (int r = lane; r < kp.bs; r += 32) items += (tiles_of(r) + c - 1) / c;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) items += __shfl_xor_sync(0xffffffffu, items, o);
+      const long long waves = ((long long)items * kp.n_kv + kp.slots - 1) / kp.slots;
+      const long long cost = waves * (kAttnPlanStartTiles + c);
+      if (best_cost < 0 || cost < best_cost || (cost == best_cost && c > best)) {
+        best_cost = cost;
+        best = c;
+        best_items = items;
+      }
+    }
+    if (lane == 0) {
+      kp.out[0] = 64 * best;   // keys per split
+      kp.out[1] = best_items;  // (request, split) items of the batch
     }
   }
   // this row's entries of the call's RoPE table (read by the QKV epilogues)
