@@ -137,8 +137,8 @@ __device__ __forceinline__ void epilogue_row_scales(const EpiParams& e, int row0
 // (0..127), scaled by rs[j] when the input rows carry a deferred norm (rs is
 // ignored otherwise); the residual epilogue overwrites it. red is a
 // [8][kChunkRows]-float scratch area (8-byte aligned). Called by 128 threads with
-// t = their tile row; the residual and argmax epilogues synchronise the 128
-// threads (named barrier 2).
+// t = their tile row; the residual, argmax and (wide) injection epilogues
+// synchronise the 128 threads (named barrier 2).
 // Each of the four epilogue warps runs alone on its scheduler. A chunk of a few
 // rows (the rows one split owns in a split-K cluster) takes a small rolled loop:
 // the code is fetched cold once per CTA and its size sets the time. Wider chunks
@@ -222,20 +222,21 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
     const int* const page_table = e.page_table;
     const int max_pages = e.max_pages, num_pages = e.num_pages, page_size = e.page_size, n_kv = e.n_kv;
     int* const status = e.status;
-    // destination of row j (-1: not stored; a bad position or page is flagged)
-    auto dest = [&](int j, int* pos_out) -> long long {
+    // destination of row j (-1: not stored; a bad position or page is flagged by
+    // the thread that has `flag`)
+    auto dest = [&](int j, int* pos_out, bool flag) -> long long {
       const int m = row0 + j;
       const int req = m / rpr, i = m % rpr;
       if (j >= nrows || (row_count && i >= __ldg(row_count + req))) return -1;
       const int ps = __ldg(pos_base + req) + i;
       const int slot = ps / page_size;
       if (ps < 0 || slot >= max_pages) {
-        if (t == 0) flag_error(status, ST_BAD_PAGE);
+        if (flag) flag_error(status, ST_BAD_PAGE);
         return -1;
       }
       const int page = __ldg(page_table + (size_t)req * max_pages + slot);
       if (page < 0 || page >= num_pages) {
-        if (t == 0) flag_error(status, ST_BAD_PAGE);
+        if (flag) flag_error(status, ST_BAD_PAGE);
         return -1;
       }
       *pos_out = ps;
@@ -245,7 +246,7 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
 #pragma unroll 1
       for (int j = 0; j < nrows; ++j) {
         int ps = 0;
-        const long long dst = dest(j, &ps);
+        const long long dst = dest(j, &ps, t == 0);
         if (dst < 0) continue;
         float v = A(j, t);
         if (rope) {
@@ -257,15 +258,24 @@ __device__ inline void epilogue_chunk_k(const EpiParams& e, int tile, int row0, 
       }
       return;
     }
+    // Wider chunks: thread t < nrows finds row t's cache slot once for all 128
+    // columns (the head's offset added per thread), through shared memory
+    long long* slot_of = reinterpret_cast<long long*>(red);   // [kChunkRows]; -1: not stored
+    if (t < nrows) {
+      int ps = 0;
+      const long long d0 = dest(t, &ps, true);   // this thread's column: head, jd
+      slot_of[t] = d0 < 0 ? -1 : d0 - ((long long)head * page_size * d + jd);
+    }
+    asm volatile("bar.sync 2, 128;" ::: "memory");
+    const long long col = (long long)head * page_size * d + jd;
 #pragma unroll 1
     for (int j0 = 0; j0 < nrows; j0 += kEpiU) {
       // destination of each row (-1: not stored), then the rotation
       long long dst[kEpiU];
-      int pos[kEpiU];
 #pragma unroll
       for (int u = 0; u < kEpiU; ++u) {
-        pos[u] = 0;
-        dst[u] = dest(j0 + u, &pos[u]);
+        const long long sl = j0 + u < nrows ? slot_of[j0 + u] : -1;
+        dst[u] = sl < 0 ? -1 : sl + col;
       }
       float2 r[kEpiU];
       if (rope) {
