@@ -300,6 +300,11 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   p.x_split = g.x_split ? 1 : 0;
   p.x_plane_rows = g.M;
   p.m_tile = std::min(g.x_split ? 128 : 256, (g.M + 15) / 16 * 16);
+  // Few output tiles at 128 rows but more than the SMs at 64: take 64, so that two
+  // CTAs share an SM and each one's epilogue runs under the other's MMAs.
+  if (g.x_split && p.m_tile == 128 && g.M > 128 && n_tiles * ((g.M + 127) / 128) <= ctx->num_sms &&
+      n_tiles * ((g.M + 63) / 64) > ctx->num_sms)
+    p.m_tile = 64;
   p.m_blocks = (g.M + p.m_tile - 1) / p.m_tile;
   // accumulator columns: the hi plane's m_tile, then the lo plane's (read 32 at a time)
   p.tmem_cols = std::max(32, pow2_at_least(p.x_split ? p.m_tile + (p.m_tile + 31) / 32 * 32 : p.m_tile));
