@@ -61,7 +61,7 @@ typedef enum {
   DFLASH_ERR_OOM = 3,          /* device workspace (dflash_create) or host allocation failed */
   DFLASH_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up */
   DFLASH_ERR_DEVICE = 5,       /* a kernel met an out-of-range id, page or position */
-  DFLASH_ERR_UNSUPPORTED = 6   /* a shape this build has no kernel for */
+  DFLASH_ERR_UNSUPPORTED = 6   /* a shape the library has no kernel for */
 } dflash_status;
 
 typedef enum { DFLASH_F32 = 0, DFLASH_BF16 = 1, DFLASH_F16 = 2 } dflash_dtype;
