@@ -300,9 +300,13 @@ dflash_status run_gemm(dflash_ctx* ctx, GemmSpec g, cudaStream_t st) {
   p.x_split = g.x_split ? 1 : 0;
   p.x_plane_rows = g.M;
   p.m_tile = std::min(g.x_split ? 128 : 256, (g.M + 15) / 16 * 16);
+  // One plane, 256-row tiles and fewer output tiles than SMs: a K split would not
+  // fit (its receive buffer takes the ring), so a few CTAs would stream everything;
+  // take 128 rows (the fusion projection at serving bs16 ran on 32 CTAs).
+  if (!g.x_split && p.m_tile == 256 && n_tiles * ((g.M + 255) / 256) <= ctx->num_sms) p.m_tile = 128;
   // Few output tiles at 128 rows but more than the SMs at 64: take 64, so that two
   // CTAs share an SM and each one's epilogue runs under the other's MMAs.
-  if (g.x_split && p.m_tile == 128 && g.M > 128 && n_tiles * ((g.M + 127) / 128) <= ctx->num_sms &&
+  if (p.m_tile == 128 && g.M > 128 && n_tiles * ((g.M + 127) / 128) <= ctx->num_sms &&
       n_tiles * ((g.M + 63) / 64) > ctx->num_sms)
     p.m_tile = 64;
   p.m_blocks = (g.M + p.m_tile - 1) / p.m_tile;
