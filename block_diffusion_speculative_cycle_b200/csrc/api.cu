@@ -985,6 +985,25 @@ dflash_status draft_impl(dflash_ctx* ctx, const int* d_anchor, const int* d_ctx_
         }
       }
       if (best >= 1e30) return DFLASH_ERR_UNSUPPORTED;
+      // A global merge chosen in the full form (long contexts, few pairs): run it in
+      // the compact form, two CTAs per SM with half the keys each (measured at the
+      // Coder-30B shape, bs 1: B 16 1340 -> 1365, B 8 1428 -> 1487 cycles/s).
+      if (ctx->attn_form < 0 && attn_gmerge && !attn_compact) {
+        const int sp_max = std::min(2 * ctx->num_sms / std::max(pairs, 1), (int)(ctx->att_rows / ((size_t)pairs * nr)));
+        double best_c = 1e30;
+        for (int sp = 2; sp <= sp_max; ++sp) {
+          int kp = (std::max(span, 1) + sp - 1) / sp;
+          kp = (kp + 63) / 64 * 64;
+          if (std::max(1, (span + kp - 1) / kp) != sp) continue;
+          const double cost = kStart + kMergeKernel + (kp / 64 + blk_tiles) * 1.25;
+          if (cost < best_c) {
+            best_c = cost;
+            n_splits = sp;
+            kps = kp;
+            attn_compact = true;
+          }
+        }
+      }
       // Many (request, KV head) pairs: the batch's contexts are usually ragged, and
       // a plan for the longest request leaves most CTA slots idle behind it. The
       // global merge then takes a split size that the device picks from the actual
