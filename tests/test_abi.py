@@ -1,6 +1,7 @@
 """Host-side checks of the C ABI that need no GPU: the library builds, loads and
 exports every entry point include/dflash.h declares, and the binding declares
 the same names."""
+import ctypes
 import os
 import re
 
@@ -129,3 +130,38 @@ def test_cycle_calls_reject_a_null_context(lib_path):
     assert lib.dflash_inject_ctx(None, None, 1, 1, None, None, None, None, None, 1, 1, None) == 1
     assert lib.dflash_draft_block(None, None, None, 1, 4, None, None, None, 1, 1, 0, None, None, None) == 1
     assert lib.dflash_get_error(None, None) == 1
+
+
+def test_loop_sampling_and_policy_calls_check_their_arguments_on_the_host(lib_path):
+    """The device-loop, sampled and acceptance-count calls refuse bad arguments with
+    DFLASH_ERR_ARG (1) before any launch, so these run without a GPU. Pointers that
+    are only checked for null are fake addresses, never dereferenced."""
+    lib = _binding.load_library(lib_path)
+    fake = ctypes.c_void_p(0x1000)
+    # a null context
+    taps = (ctypes.c_int * 1)(0)
+    assert lib.dflash_target_forward(None, fake, None, None, 1, 1, fake, None, None, fake, 1, 1, 0, taps, 0, fake,
+                                     None, None) == 1
+    assert lib.dflash_draft_block_sample(None, fake, fake, 1, 4, None, None, fake, 1, 1, 0, ctypes.c_float(1.0), 7,
+                                         fake, fake, None, None) == 1
+    # the commit: empty batch, or drafts missing for B > 1
+    args = [fake, fake, fake, fake, 8, fake, fake, fake, fake, fake, None]
+    assert lib.dflash_spec_commit(0, 4, *args) == 1
+    assert lib.dflash_spec_commit(1, 4, None, *args[1:]) == 1
+    # sampled verify: temperature, empty batch, misaligned workspace
+    ws_bytes = lib.dflash_verify_sampled_workspace_size(2, 4, 1000)
+    assert ws_bytes > 0
+    good_ws = ctypes.c_void_p(0x100000)
+
+    def vs(bs, temp, ws):
+        return lib.dflash_verify_sampled(fake, _binding.DFLASH_F32, fake, fake, bs, 4, 1000, ctypes.c_float(temp), fake,
+                                         fake, fake, fake, ws, ws_bytes, None)
+
+    assert vs(2, 0.0, good_ws) == 1
+    assert vs(2, float("inf"), good_ws) == 1
+    assert vs(0, 1.0, good_ws) == 1
+    assert vs(2, 1.0, ctypes.c_void_p(0x100010)) == 1
+    # acceptance counts: null arrays, a block past the count array; B = 1 tests nothing
+    assert lib.dflash_acceptance_count(None, 2, 4, fake, 16, None) == 1
+    assert lib.dflash_acceptance_count(fake, 2, 17, fake, 16, None) == 1
+    assert lib.dflash_acceptance_count(fake, 2, 1, fake, 16, None) == 0
